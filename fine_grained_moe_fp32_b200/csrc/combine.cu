@@ -1,0 +1,79 @@
+// Combine: weighted un-permute of the routed expert outputs plus the shared
+// experts (dots.llm1 Technical Report, Method: shared experts are always on;
+// the routed experts enter with their gate weights).
+//
+//   y[t] = y_shared[t] + sum_{j < k} w[t, j] * y_perm[row_of[t*k + j]]
+//
+// fp32 accumulation, slot j in ascending order, one rounding to bf16.  One CTA
+// per token; 16-byte vectors (8 bf16) along the hidden dimension.
+#include <cuda_bf16.h>
+
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kMaxK = 8;
+
+__device__ __forceinline__ void add_bf16x8(float (&acc)[8], uint4 v, float w) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[2 * i] = fmaf(w, __uint_as_float(u[i] << 16), acc[2 * i]);
+    acc[2 * i + 1] = fmaf(w, __uint_as_float(u[i] & 0xFFFF0000u), acc[2 * i + 1]);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+combine_kernel(const uint16_t* __restrict__ y_perm, const int32_t* __restrict__ row_of,
+               const float* __restrict__ topk_w, const float* __restrict__ y_shared,
+               uint16_t* __restrict__ y, int d, int k, int64_t cap) {
+  const int t = blockIdx.x;
+  __shared__ int rows[kMaxK];
+  __shared__ float ws[kMaxK];
+  if (threadIdx.x < k) {
+    const int r = row_of[(size_t)t * k + threadIdx.x];
+    rows[threadIdx.x] = (r >= 0 && r < cap) ? r : -1;
+    ws[threadIdx.x] = topk_w[(size_t)t * k + threadIdx.x];
+  }
+  __syncthreads();
+  const int nv = d / 8;
+  for (int v = threadIdx.x; v < nv; v += kThreads) {
+    float acc[8];
+    if (y_shared != nullptr) {
+      const float4* s = reinterpret_cast<const float4*>(y_shared + (size_t)t * d) + 2 * v;
+      const float4 a = s[0], b = s[1];
+      acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
+      acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    }
+    for (int j = 0; j < k; ++j) {
+      if (rows[j] < 0) continue;
+      const uint4 val = reinterpret_cast<const uint4*>(y_perm + (size_t)rows[j] * d)[v];
+      add_bf16x8(acc, val, ws[j]);
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * i]));
+      const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * i + 1]));
+      o[i] = lo | (hi << 16);
+    }
+    reinterpret_cast<uint4*>(y + (size_t)t * d)[v] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const Shape& s, const uint16_t* y_perm, const int32_t* row_of,
+                           const float* topk_w, const float* y_shared, uint16_t* y,
+                           cudaStream_t st) {
+  if (s.T == 0) return cudaSuccess;
+  combine_kernel<<<s.T, kThreads, 0, st>>>(y_perm, row_of, topk_w, y_shared, y, s.d, s.k, s.cap);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,536 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05, sm_100a).
+//
+// dots.llm1 Technical Report, Key claims / Method (systems paragraph): the
+// grouped GEMM pads each expert's token segment to a multiple of the MMA tile
+// so that every tile holds one expert and scheduling looks like a plain GEMM.
+// The pages' kernel targets Hopper WGMMA; this is a Blackwell design:
+//
+//  * swap-AB: the expert WEIGHTS are the M = 128 operand, the TOKENS of a
+//    segment are the N operand (N = 16..256 in steps of 16), so a segment only
+//    needs padding to 16 rows and decode-sized segments stream weights at full
+//    MMA width;
+//  * gate/up fusion: the A tile of the gate/up GEMM stacks 64 rows of W1 over
+//    the same 64 rows of W3, so one MMA per K-step yields both, and SwiGLU runs
+//    in the epilogue (gate lanes 0-63, up lanes 64-127, exchanged via smem);
+//  * persistent CTAs (one per SM) walk a static tile list computed on the
+//    device from the segment offsets (group-major, token tile, feature tile
+//    fastest so concurrent CTAs share the weight and token tiles in L2);
+//  * warp roles: warp 0 issues TMA loads into a STAGES-deep smem ring, warp 1
+//    issues tcgen05.mma into one of two TMEM accumulators, warps 2-5 drain
+//    the other accumulator (tcgen05.ld) and store;
+//  * every pipeline wait is bounded: on expiry the CTA records a timeout in
+//    the status word, drains its in-flight copies, frees TMEM and returns.
+//
+// The shared experts ride along as one extra group: for the gate/up GEMM the
+// S shared experts are one expert of S*I features over all T tokens (read
+// from x); for the down GEMM their K dimension is the concatenation of the S
+// experts (a 3-D tensor map walks the planes), so y_shared is their sum.
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include "moe_internal.h"
+#include "ptx_sm100.cuh"
+
+namespace moe {
+namespace {
+
+enum Mode : int { kSwiGLU = 0, kDown = 1 };
+
+constexpr int kBK = 64;            // K elements per stage: one 128-byte swizzle row
+constexpr int kBoxB = 32;          // token rows per TMA box of the B operand
+constexpr int kABytes = 128 * 128; // A stage: 128 rows x 128 bytes
+constexpr int kMaxGroups = 129;    // 128 routed experts + the shared group
+constexpr int kThreads = 192;      // 6 warps
+constexpr int kEpiThreads = 128;
+constexpr uint64_t kDrainLimitNs = 1000000000ull;
+
+struct GemmParams {
+  int E;                // routed groups
+  int has_shared;       // 1: group E = shared experts over T rows
+  int T;
+  int ft_routed;        // feature tiles of a routed group
+  int ft_shared;        // feature tiles of the shared group
+  int kit_routed;       // K iterations (of 64) of a routed group
+  int kit_shared;       // K iterations of the shared group
+  int k_plane;          // K extent of one plane of the A map (down GEMM: I)
+  int a_rows_group;     // A-map rows per routed group (gate/up: I, down: d)
+  int a_evict_first;    // stream weights with L2 evict_first (decode)
+  const int32_t* offsets;
+  void* out_routed;
+  int ld_routed;
+  void* out_shared;
+  int ld_shared;
+  int shared_f32;
+  unsigned int* status;
+  uint64_t wait_limit_ns;
+};
+
+struct TileInfo {
+  int g, ft, row0, nrows, nmma, kit;
+};
+
+struct SmemCtl {
+  uint64_t full[16];
+  uint64_t empty[16];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int ngroups;
+  int total_tiles;
+  int prefix[kMaxGroups + 1];
+  int row0[kMaxGroups];
+  int rows[kMaxGroups];
+};
+
+template <int NT>
+__device__ __forceinline__ TileInfo decode_tile(const SmemCtl& c, const GemmParams& p, int tile) {
+  int lo = 0, hi = c.ngroups - 1;
+  while (lo < hi) {  // largest g with prefix[g] <= tile
+    const int mid = (lo + hi + 1) >> 1;
+    if (c.prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  TileInfo ti;
+  ti.g = lo;
+  const bool routed = lo < p.E;
+  const int nft = routed ? p.ft_routed : p.ft_shared;
+  const int local = tile - c.prefix[lo];
+  const int tt = local / nft;
+  ti.ft = local - tt * nft;
+  ti.row0 = c.row0[lo] + tt * NT;
+  ti.nrows = min(NT, c.rows[lo] - tt * NT);
+  ti.nmma = (ti.nrows + 15) & ~15;
+  ti.kit = routed ? p.kit_routed : p.kit_shared;
+  return ti;
+}
+
+__device__ __forceinline__ bool aborted(const SmemCtl& c) {
+  return *reinterpret_cast<const volatile int*>(&c.abort_flag) != 0;
+}
+
+__device__ __forceinline__ void record_timeout(SmemCtl& c, const GemmParams& p) {
+  *reinterpret_cast<volatile int*>(&c.abort_flag) = 1;
+  if (p.status != nullptr) atomicCAS(p.status, 0u, (unsigned)DEV_TIMEOUT);
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+
+template <int MODE, int NT, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r,
+                    const __grid_constant__ CUtensorMap tmA2_r,
+                    const __grid_constant__ CUtensorMap tmB_r,
+                    const __grid_constant__ CUtensorMap tmA_s,
+                    const __grid_constant__ CUtensorMap tmA2_s,
+                    const __grid_constant__ CUtensorMap tmB_s, const GemmParams p) {
+  constexpr int kBBytes = NT * 128;
+  constexpr int kStageBytes = kABytes + kBBytes;
+  constexpr uint32_t kTmemCols = (2 * NT < 32) ? 32 : 2 * NT;
+
+  __shared__ SmemCtl ctl;
+  extern __shared__ uint8_t dsmem_raw[];
+  const uint32_t raw = smem_u32(dsmem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* dsmem = dsmem_raw + (sbase - raw);
+  float* up_buf = reinterpret_cast<float*>(dsmem + STAGES * kStageBytes);  // [32][64]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- setup: tile table, barriers, TMEM
+  if (warp == 0) {
+    const int G = p.E + (p.has_shared ? 1 : 0);
+    // each lane handles groups [lane*5, lane*5 + 5): 160 >= kMaxGroups
+    int local[5];
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+      const int g = lane * 5 + i;
+      int tiles = 0;
+      if (g < G) {
+        int r0, nr, nft;
+        if (g < p.E) {
+          r0 = p.offsets[g];
+          nr = p.offsets[g + 1] - r0;
+          nft = p.ft_routed;
+        } else {
+          r0 = 0;
+          nr = p.T;
+          nft = p.ft_shared;
+        }
+        if (nr < 0) nr = 0;
+        ctl.row0[g] = r0;
+        ctl.rows[g] = nr;
+        tiles = (int)ceil_div(nr, NT) * nft;
+      }
+      local[i] = tiles;
+      sum += tiles;
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+      const int g = lane * 5 + i;
+      if (g < G) ctl.prefix[g] = run;
+      run += local[i];
+    }
+    if (lane == 31) {
+      ctl.prefix[G] = incl;
+      ctl.total_tiles = incl;
+      ctl.ngroups = G;
+    }
+    if (lane == 0) {
+      for (int s = 0; s < STAGES; ++s) {
+        mbar_init(smem_u32(&ctl.full[s]), 1);
+        mbar_init(smem_u32(&ctl.empty[s]), 1);
+      }
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(smem_u32(&ctl.tfull[b]), 1);
+        mbar_init(smem_u32(&ctl.tempty[b]), kEpiThreads);
+      }
+      mbar_init(smem_u32(&ctl.drain), 1);
+      ctl.abort_flag = 0;
+      fence_mbar_init();
+      prefetch_tmap(&tmA_r);
+      prefetch_tmap(&tmB_r);
+      if (MODE == kSwiGLU) prefetch_tmap(&tmA2_r);
+    }
+  } else if (warp == 1) {
+    tmem_alloc(smem_u32(&ctl.tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = ctl.tmem_base;
+  const int total = ctl.total_tiles;
+
+  if (warp == 0) {
+    // ================= TMA producer =================
+    if (lane == 0) {
+      const uint64_t pol_a = p.a_evict_first ? policy_evict_first() : policy_evict_normal();
+      const uint64_t pol_b = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t filled = 0;       // bit s: stage s was filled at least once
+      uint32_t fill_parity = 0;  // bit s: parity of the phase of the last fill of s
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const TileInfo ti = decode_tile<NT>(ctl, p, tile);
+        const bool routed = ti.g < p.E;
+        const CUtensorMap* tA = routed ? &tmA_r : &tmA_s;
+        const CUtensorMap* tA2 = routed ? &tmA2_r : &tmA2_s;
+        const CUtensorMap* tB = routed ? &tmB_r : &tmB_s;
+        const int nbox = (ti.nmma + kBoxB - 1) / kBoxB;
+        const uint32_t tx = kABytes + nbox * kBoxB * 128;
+        const int arow = MODE == kSwiGLU ? (routed ? ti.g * p.a_rows_group : 0) + ti.ft * 64
+                                         : (routed ? ti.g * p.a_rows_group : 0) + ti.ft * 128;
+        for (int kc = 0; kc < ti.kit; ++kc) {
+          if (aborted(ctl)) { ok = false; break; }
+          if (!mbar_wait_bounded(smem_u32(&ctl.empty[stage]), phase ^ 1u, p.wait_limit_ns)) {
+            record_timeout(ctl, p);
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&ctl.full[stage]);
+          mbar_arrive_expect_tx(fb, tx);
+          const uint32_t sA = sbase + stage * kStageBytes;
+          const uint32_t sB = sA + kABytes;
+          const int kk = kc * kBK;
+          if (MODE == kSwiGLU) {
+            tma_load_3d(sA, tA, fb, kk, arow, 0, pol_a);
+            tma_load_3d(sA + kABytes / 2, tA2, fb, kk, arow, 0, pol_a);
+          } else {
+            const int plane = kk / p.k_plane;
+            tma_load_3d(sA, tA, fb, kk - plane * p.k_plane, arow, plane, pol_a);
+          }
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d(sB + b * kBoxB * 128, tB, fb, kk, ti.row0 + b * kBoxB, pol_b);
+          filled |= 1u << stage;
+          fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // drain: every fill this thread issued must land before the CTA exits
+      for (int s = 0; s < STAGES; ++s) {
+        if (((filled >> s) & 1u) &&
+            !mbar_wait_bounded(smem_u32(&ctl.full[s]), (fill_parity >> s) & 1u, kDrainLimitNs))
+          record_timeout(ctl, p);
+      }
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const TileInfo ti = decode_tile<NT>(ctl, p, tile);
+        const uint32_t idesc = idesc_bf16_f32_m128((uint32_t)ti.nmma);
+        if (aborted(ctl) ||
+            !mbar_wait_bounded(smem_u32(&ctl.tempty[acc]), acc_phase ^ 1u, p.wait_limit_ns)) {
+          if (!aborted(ctl)) record_timeout(ctl, p);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dt = tmem_base + (uint32_t)(acc * NT);
+        for (int kc = 0; kc < ti.kit; ++kc) {
+          if (aborted(ctl) ||
+              !mbar_wait_bounded(smem_u32(&ctl.full[stage]), phase, p.wait_limit_ns)) {
+            if (!aborted(ctl)) record_timeout(ctl, p);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sA = sbase + stage * kStageBytes;
+          const uint32_t sB = sA + kABytes;
+#pragma unroll
+          for (int k4 = 0; k4 < kBK / 16; ++k4) {
+            const uint64_t ad = sdesc_kmajor_sw128(sA + k4 * 32);
+            const uint64_t bd = sdesc_kmajor_sw128(sB + k4 * 32);
+            mma_bf16_ss(dt, ad, bd, idesc, (kc | k4) != 0 ? 1u : 0u);
+          }
+          mma_commit(smem_u32(&ctl.empty[stage]));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(&ctl.tfull[acc]));
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      // drain: all MMAs issued by this thread complete before TMEM is freed
+      mma_commit(smem_u32(&ctl.drain));
+      if (!mbar_wait_bounded(smem_u32(&ctl.drain), 0, kDrainLimitNs)) record_timeout(ctl, p);
+    }
+  } else {
+    // ================= epilogue (warps 2..5) =================
+    const int q = warp & 3;             // TMEM lane quarter this warp may access
+    const int frow = q * 32 + lane;     // accumulator row = TMEM lane
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      const TileInfo ti = decode_tile<NT>(ctl, p, tile);
+      // the four epilogue warps decide together, so that none of them is left
+      // waiting on a named barrier the others have abandoned
+      bool bad = aborted(ctl);
+      if (!bad && !mbar_wait_bounded(smem_u32(&ctl.tfull[acc]), acc_phase, p.wait_limit_ns)) {
+        record_timeout(ctl, p);
+        bad = true;
+      }
+      if (bar_red_or(2, kEpiThreads, bad)) break;
+      tc_fence_after();
+      const bool routed = ti.g < p.E;
+      const uint32_t tbase = tmem_base + (uint32_t)(acc * NT) + ((uint32_t)(q * 32) << 16);
+      for (int c0 = 0; c0 < ti.nrows; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tbase + (uint32_t)c0, v);
+        tmem_ld_wait();
+        const int nj = min(32, ti.nrows - c0);
+        if (MODE == kDown) {
+          const int col = ti.ft * 128 + frow;
+          if (routed) {
+            uint16_t* out = static_cast<uint16_t*>(p.out_routed);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (j < nj)
+                out[(size_t)(ti.row0 + c0 + j) * p.ld_routed + col] =
+                    __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+            }
+          } else if (p.shared_f32) {
+            float* out = static_cast<float*>(p.out_shared);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nj) out[(size_t)(ti.row0 + c0 + j) * p.ld_shared + col] = __uint_as_float(v[j]);
+          } else {
+            uint16_t* out = static_cast<uint16_t*>(p.out_shared);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nj)
+                out[(size_t)(ti.row0 + c0 + j) * p.ld_shared + col] =
+                    __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+          }
+        } else {
+          // lanes 64..127 hold W3 x (up), lanes 0..63 hold W1 x (gate)
+          if (q >= 2) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) up_buf[j * 64 + (frow - 64)] = __uint_as_float(v[j]);
+          }
+          named_bar_sync(1, kEpiThreads);
+          if (q < 2) {
+            uint16_t* out = static_cast<uint16_t*>(routed ? p.out_routed : p.out_shared);
+            const int ld = routed ? p.ld_routed : p.ld_shared;
+            const int col = ti.ft * 64 + frow;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (j < nj) {
+                const float g = __uint_as_float(v[j]);
+                const float h = silu_f(g) * up_buf[j * 64 + frow];
+                out[(size_t)(ti.row0 + c0 + j) * ld + col] =
+                    __bfloat16_as_ushort(__float2bfloat16_rn(h));
+              }
+            }
+          }
+          named_bar_sync(1, kEpiThreads);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&ctl.tempty[acc]));
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// bf16 tensor viewed as (inner, rows, planes), box (64, box_rows, 1), 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t planes,
+              uint32_t box_rows, int rank) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {inner, rows, planes};
+  cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+  cuuint32_t box[3] = {(cuuint32_t)kBK, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  if (rows == 0) dims[1] = 1;  // an empty operand is never read; keep the map valid
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+                  dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int MODE, int NT, int STAGES>
+cudaError_t launch_one(const CUtensorMap* maps, const GemmParams& p, int num_sms,
+                       cudaStream_t st) {
+  constexpr int kBBytes = NT * 128;
+  constexpr size_t smem = (size_t)STAGES * (kABytes + kBBytes) + 32 * 64 * 4 + 1024;
+  static_assert(STAGES <= 16, "barrier arrays hold 16 stages");
+  static_assert(smem + sizeof(SmemCtl) <= 232448, "shared memory budget");
+  auto kern = grouped_gemm_kernel<MODE, NT, STAGES>;
+  cudaError_t err =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  kern<<<num_sms, kThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_gemms(const Shape& s, const GroupedGemmArgs& a, int num_sms,
+                                 unsigned int* status, uint64_t wait_limit_ns, cudaStream_t st,
+                                 cudaEvent_t between) {
+  const bool shared = s.S > 0 && a.x != nullptr && a.ws1 != nullptr && a.ws3 != nullptr &&
+                      a.ws2 != nullptr && a.h_shared != nullptr && a.y_shared != nullptr &&
+                      s.T > 0;
+  const bool small = (int64_t)s.T * s.k <= (int64_t)24 * s.E;  // decode-sized segments
+  const uint32_t boxB = kBoxB;
+  CUtensorMap m[6];
+  // ---- gate/up GEMM + SwiGLU
+  {
+    bool ok = make_map(&m[0], a.w1, s.d, (uint64_t)s.E * s.I, 1, 64, 3) &&
+              make_map(&m[1], a.w3, s.d, (uint64_t)s.E * s.I, 1, 64, 3) &&
+              make_map(&m[2], a.x_perm, s.d, s.cap, 1, boxB, 2);
+    if (shared) {
+      ok = ok && make_map(&m[3], a.ws1, s.d, (uint64_t)s.S * s.I, 1, 64, 3) &&
+           make_map(&m[4], a.ws3, s.d, (uint64_t)s.S * s.I, 1, 64, 3) &&
+           make_map(&m[5], a.x, s.d, s.T, 1, boxB, 2);
+    } else {
+      m[3] = m[0];
+      m[4] = m[1];
+      m[5] = m[2];
+    }
+    if (!ok) return cudaErrorInvalidValue;
+    GemmParams p{};
+    p.E = s.E;
+    p.has_shared = shared ? 1 : 0;
+    p.T = s.T;
+    p.ft_routed = s.I / 64;
+    p.ft_shared = s.S * s.I / 64;
+    p.kit_routed = s.d / kBK;
+    p.kit_shared = s.d / kBK;
+    p.k_plane = s.d;
+    p.a_rows_group = s.I;
+    p.a_evict_first = small ? 1 : 0;
+    p.offsets = a.offsets;
+    p.out_routed = a.h_perm;
+    p.ld_routed = s.I;
+    p.out_shared = a.h_shared;
+    p.ld_shared = s.S * s.I;
+    p.shared_f32 = 0;
+    p.status = status;
+    p.wait_limit_ns = wait_limit_ns;
+    cudaError_t err = small ? launch_one<kSwiGLU, 32, 10>(m, p, num_sms, st)
+                            : launch_one<kSwiGLU, 256, 4>(m, p, num_sms, st);
+    if (err != cudaSuccess) return err;
+    if (between != nullptr && (err = cudaEventRecord(between, st)) != cudaSuccess) return err;
+  }
+  // ---- down GEMM
+  {
+    bool ok = make_map(&m[0], a.w2, s.I, (uint64_t)s.E * s.d, 1, 128, 3) &&
+              make_map(&m[2], a.h_perm, s.I, s.cap, 1, boxB, 2);
+    m[1] = m[0];
+    if (shared) {
+      ok = ok && make_map(&m[3], a.ws2, s.I, s.d, s.S, 128, 3) &&
+           make_map(&m[5], a.h_shared, (uint64_t)s.S * s.I, s.T, 1, boxB, 2);
+      m[4] = m[3];
+    } else {
+      m[3] = m[0];
+      m[4] = m[1];
+      m[5] = m[2];
+    }
+    if (!ok) return cudaErrorInvalidValue;
+    GemmParams p{};
+    p.E = s.E;
+    p.has_shared = shared ? 1 : 0;
+    p.T = s.T;
+    p.ft_routed = s.d / 128;
+    p.ft_shared = s.d / 128;
+    p.kit_routed = s.I / kBK;
+    p.kit_shared = s.S * s.I / kBK;
+    p.k_plane = s.I;
+    p.a_rows_group = s.d;
+    p.a_evict_first = small ? 1 : 0;
+    p.offsets = a.offsets;
+    p.out_routed = a.y_perm;
+    p.ld_routed = s.d;
+    p.out_shared = a.y_shared;
+    p.ld_shared = s.d;
+    p.shared_f32 = 1;
+    p.status = status;
+    p.wait_limit_ns = wait_limit_ns;
+    cudaError_t err = small ? launch_one<kDown, 32, 10>(m, p, num_sms, st)
+                            : launch_one<kDown, 256, 4>(m, p, num_sms, st);
+    if (err != cudaSuccess) return err;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace moe

@@ -1,0 +1,340 @@
+// C ABI of the library: argument checks, workspace layout and the launch
+// sequence of every entry point declared in include/moe_b200.h.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe_b200.h"
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+// First device-side error since the last moe_get_last_device_status().
+__device__ unsigned int g_device_status = 0;
+
+constexpr int kMaxDevices = 64;
+constexpr int kPlanSMs = 148;  // split-K planning of the router is device independent
+constexpr uint64_t kDefaultWaitNs = 1000000000ull;
+uint64_t g_wait_limit_ns = kDefaultWaitNs;
+cudaEvent_t g_phase_events[6] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+bool g_phase_on = false;
+
+cudaError_t phase(int i, cudaStream_t st) {
+  return g_phase_on ? cudaEventRecord(g_phase_events[i], st) : cudaSuccess;
+}
+
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+  unsigned int* status = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+const DeviceInfo* device_info() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return nullptr;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    d.status = static_cast<unsigned int*>(p);
+    d.ready = true;
+  }
+  return &d;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_dims(const moe_dims* dims, Shape* s) {
+  if (dims == nullptr) return MOE_ERR_INVALID_ARG;
+  const moe_dims& m = *dims;
+  if (m.T < 0 || m.d <= 0 || m.E <= 0 || m.k <= 0 || m.I <= 0 || m.n_shared < 0 || m.align <= 0)
+    return MOE_ERR_INVALID_ARG;
+  if (m.E > 128 || m.k > m.E || m.k > 8 || m.d % 128 != 0 || m.I % 64 != 0 || m.align % 16 != 0 ||
+      m.n_shared > 4)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  const int64_t cap = (int64_t)m.T * m.k + (int64_t)m.E * (m.align - 1);
+  if (cap >= (int64_t)INT32_MAX / 2 || (int64_t)m.T * m.k >= INT32_MAX / 2)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  *s = Shape{m.T, m.d, m.E, m.k, m.I, m.n_shared, m.align, cap};
+  return MOE_OK;
+}
+
+size_t al256(size_t b) { return (b + 255) & ~size_t(255); }
+
+moe_ws_layout make_layout(const Shape& s) {
+  moe_ws_layout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += al256(bytes);
+    return at;
+  };
+  L.route_partials = take(router_partials_bytes(s, kPlanSMs));
+  L.probs = take((size_t)s.T * s.E * 4);
+  L.topk_idx = take((size_t)s.T * s.k * 4);
+  L.topk_w = take((size_t)s.T * s.k * 4);
+  L.counts = take((size_t)s.E * 4);
+  L.offsets = take((size_t)(s.E + 1) * 4);
+  L.row_of = take((size_t)s.T * s.k * 4);
+  L.token_of_row = take((size_t)s.cap * 4);
+  L.permute_scratch = take(permute_scratch_bytes(s));
+  L.x_perm = take((size_t)s.cap * s.d * 2);
+  L.h_perm = take((size_t)s.cap * s.I * 2);
+  L.y_perm = take((size_t)s.cap * s.d * 2);
+  L.h_shared = take((size_t)s.T * s.S * s.I * 2);
+  L.y_shared = take((size_t)s.T * s.d * 4);
+  L.total = off;
+  return L;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+template <typename T>
+T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(base) + off);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int64_t moe_capacity(const moe_dims* dims) {
+  Shape s;
+  if (check_dims(dims, &s) != MOE_OK) return 0;
+  return s.cap;
+}
+
+const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOE_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_TIMEOUT: return "a bounded device wait ran out";
+    default: return "unknown status";
+  }
+}
+
+size_t moe_route_workspace_size(const moe_dims* dims) {
+  Shape s;
+  if (check_dims(dims, &s) != MOE_OK) return 0;
+  return al256(router_partials_bytes(s, kPlanSMs));
+}
+
+int moe_route(const moe_dims* dims, const moe_bf16* x, const float* w_gate, const float* bias,
+              float* probs, int32_t* topk_idx, float* topk_w, void* workspace,
+              size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != MOE_OK) return rc;
+  if (s.T == 0) return MOE_OK;
+  if (x == nullptr || w_gate == nullptr || topk_idx == nullptr || topk_w == nullptr ||
+      !aligned(x, 16) || !aligned(w_gate, 16))
+    return MOE_ERR_INVALID_ARG;
+  const size_t need = router_partials_bytes(s, kPlanSMs);
+  if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256))
+    return MOE_ERR_WORKSPACE;
+  if (device_info() == nullptr) return MOE_ERR_CUDA;
+  return cuda_status(launch_router(s, x, w_gate, bias, probs, topk_idx, topk_w,
+                                   static_cast<float*>(workspace), kPlanSMs,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_permute_workspace_size(const moe_dims* dims) {
+  Shape s;
+  if (check_dims(dims, &s) != MOE_OK) return 0;
+  return al256(permute_scratch_bytes(s));
+}
+
+int moe_permute(const moe_dims* dims, const int32_t* topk_idx, const moe_bf16* x, int32_t* counts,
+                int32_t* offsets, int32_t* row_of, int32_t* token_of_row, moe_bf16* x_perm,
+                void* workspace, size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != MOE_OK) return rc;
+  if (counts == nullptr || offsets == nullptr || token_of_row == nullptr || x_perm == nullptr ||
+      (s.T > 0 && (topk_idx == nullptr || x == nullptr || row_of == nullptr)) ||
+      !aligned(x, 16) || !aligned(x_perm, 16))
+    return MOE_ERR_INVALID_ARG;
+  const size_t need = permute_scratch_bytes(s);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)))
+    return MOE_ERR_WORKSPACE;
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return MOE_ERR_CUDA;
+  return cuda_status(launch_permute(s, topk_idx, x, counts, offsets, row_of, token_of_row, x_perm,
+                                    workspace, di->status, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_grouped_swiglu(const moe_dims* dims, const moe_bf16* x_perm, const int32_t* offsets,
+                       const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
+                       moe_bf16* h_perm, moe_bf16* y_perm, void* stream) {
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != MOE_OK) return rc;
+  if (x_perm == nullptr || offsets == nullptr || w1 == nullptr || w3 == nullptr || w2 == nullptr ||
+      h_perm == nullptr || y_perm == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(x_perm, 16) || !aligned(w1, 16) || !aligned(w3, 16) || !aligned(w2, 16) ||
+      !aligned(h_perm, 16) || !aligned(y_perm, 16))
+    return MOE_ERR_INVALID_ARG;
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return MOE_ERR_CUDA;
+  GroupedGemmArgs a{};
+  a.x_perm = x_perm;
+  a.offsets = offsets;
+  a.w1 = w1;
+  a.w3 = w3;
+  a.w2 = w2;
+  a.h_perm = h_perm;
+  a.y_perm = y_perm;
+  return cuda_status(launch_grouped_gemms(s, a, di->num_sms, di->status, g_wait_limit_ns,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int moe_combine(const moe_dims* dims, const moe_bf16* y_perm, const int32_t* row_of,
+                const float* topk_w, const float* y_shared, moe_bf16* y, void* stream) {
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != MOE_OK) return rc;
+  if (s.T == 0) return MOE_OK;
+  if (y_perm == nullptr || row_of == nullptr || topk_w == nullptr || y == nullptr ||
+      !aligned(y_perm, 16) || !aligned(y, 16) || (y_shared != nullptr && !aligned(y_shared, 16)))
+    return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_combine(s, y_perm, row_of, topk_w, y_shared, y,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_workspace_size(const moe_dims* dims) {
+  Shape s;
+  if (check_dims(dims, &s) != MOE_OK) return 0;
+  return make_layout(s).total;
+}
+
+int moe_forward_layout(const moe_dims* dims, moe_ws_layout* layout) {
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != MOE_OK) return rc;
+  if (layout == nullptr) return MOE_ERR_INVALID_ARG;
+  *layout = make_layout(s);
+  return MOE_OK;
+}
+
+int moe_forward(const moe_dims* dims, const moe_bf16* x, const float* w_gate, const float* bias,
+                const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2, const moe_bf16* ws1,
+                const moe_bf16* ws3, const moe_bf16* ws2, moe_bf16* y, void* workspace,
+                size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != MOE_OK) return rc;
+  if (w_gate == nullptr || w1 == nullptr || w3 == nullptr || w2 == nullptr ||
+      (s.T > 0 && (x == nullptr || y == nullptr)))
+    return MOE_ERR_INVALID_ARG;
+  if (s.S > 0 && (ws1 == nullptr || ws3 == nullptr || ws2 == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(w_gate, 16) || !aligned(w1, 16) || !aligned(w3, 16) ||
+      !aligned(w2, 16) || !aligned(y, 16) || !aligned(ws1, 16) || !aligned(ws3, 16) ||
+      !aligned(ws2, 16))
+    return MOE_ERR_INVALID_ARG;
+  const moe_ws_layout L = make_layout(s);
+  if (workspace == nullptr || workspace_bytes < L.total || !aligned(workspace, 256))
+    return MOE_ERR_WORKSPACE;
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+
+  float* probs = at<float>(ws, L.probs);
+  int32_t* idx = at<int32_t>(ws, L.topk_idx);
+  float* wts = at<float>(ws, L.topk_w);
+  int32_t* counts = at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* row_of = at<int32_t>(ws, L.row_of);
+  int32_t* tor = at<int32_t>(ws, L.token_of_row);
+  uint16_t* x_perm = at<uint16_t>(ws, L.x_perm);
+  uint16_t* h_perm = at<uint16_t>(ws, L.h_perm);
+  uint16_t* y_perm = at<uint16_t>(ws, L.y_perm);
+  uint16_t* h_sh = at<uint16_t>(ws, L.h_shared);
+  float* y_sh = at<float>(ws, L.y_shared);
+
+  cudaError_t e = phase(0, st);
+  if (e == cudaSuccess)
+    e = launch_router(s, x, w_gate, bias, probs, idx, wts, at<float>(ws, L.route_partials),
+                      kPlanSMs, st);
+  if (e == cudaSuccess) e = phase(1, st);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  e = launch_permute(s, idx, x, counts, offsets, row_of, tor, x_perm,
+                     at<void>(ws, L.permute_scratch), di->status, st);
+  if (e == cudaSuccess) e = phase(2, st);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  GroupedGemmArgs a{};
+  a.x_perm = x_perm;
+  a.offsets = offsets;
+  a.w1 = w1;
+  a.w3 = w3;
+  a.w2 = w2;
+  a.h_perm = h_perm;
+  a.y_perm = y_perm;
+  if (s.S > 0) {
+    a.x = x;
+    a.ws1 = ws1;
+    a.ws3 = ws3;
+    a.ws2 = ws2;
+    a.h_shared = h_sh;
+    a.y_shared = y_sh;
+  }
+  e = launch_grouped_gemms(s, a, di->num_sms, di->status, g_wait_limit_ns, st,
+                           g_phase_on ? g_phase_events[3] : nullptr);
+  if (e == cudaSuccess) e = phase(4, st);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  e = launch_combine(s, y_perm, row_of, wts, s.S > 0 ? y_sh : nullptr, y, st);
+  if (e == cudaSuccess) e = phase(5, st);
+  return cuda_status(e);
+}
+
+int moe_get_last_device_status(void* stream) {
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpy(&v, di->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpy(di->status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  switch (v) {
+    case DEV_OK: return MOE_OK;
+    case DEV_BAD_EXPERT_ID: return MOE_ERR_INVALID_ARG;
+    case DEV_TIMEOUT: return MOE_ERR_TIMEOUT;
+    default: return MOE_ERR_CUDA;
+  }
+}
+
+int moe_set_phase_events(void* const* events, int n) {
+  if (events == nullptr || n == 0) {
+    g_phase_on = false;
+    return MOE_OK;
+  }
+  if (n < 6) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < 6; ++i) {
+    if (events[i] == nullptr) return MOE_ERR_INVALID_ARG;
+    g_phase_events[i] = static_cast<cudaEvent_t>(events[i]);
+  }
+  g_phase_on = true;
+  return MOE_OK;
+}
+
+int moe_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns = ns == 0 ? kDefaultWaitNs : ns;
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,67 @@
+// Host-side declarations shared by the translation units of the library.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+// Device-side error codes written into the per-device status word (the first
+// non-zero code wins; the host maps them to the public MOE_ERR_* values).
+enum DevStatus : unsigned int {
+  DEV_OK = 0,
+  DEV_BAD_EXPERT_ID = 1,
+  DEV_TIMEOUT = 2,
+};
+
+__host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+__host__ __device__ inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+struct Shape {
+  int T, d, E, k, I, S, align;
+  int64_t cap;  // T*k + E*(align-1)
+};
+
+// ---- router (router.cu)
+constexpr int kRouterBT = 128;  // tokens per CTA tile
+constexpr int kRouterBK = 16;   // k-chunk staged in shared memory
+int router_splits(const Shape& s, int num_sms);
+size_t router_partials_bytes(const Shape& s, int num_sms);
+cudaError_t launch_router(const Shape& s, const uint16_t* x, const float* w_gate,
+                          const float* bias, float* probs, int32_t* topk_idx, float* topk_w,
+                          float* partials, int num_sms, cudaStream_t st);
+
+// ---- permutation (permute.cu)
+constexpr int kChunkTokens = 256;  // tokens per CTA in the count / scatter kernels
+size_t permute_scratch_bytes(const Shape& s);
+cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16_t* x,
+                           int32_t* counts, int32_t* offsets, int32_t* row_of,
+                           int32_t* token_of_row, uint16_t* x_perm, void* scratch,
+                           unsigned int* status, cudaStream_t st);
+
+// ---- grouped GEMMs (grouped_gemm.cu)
+struct GroupedGemmArgs {
+  // routed experts
+  const uint16_t* x_perm;  // [cap, d]
+  const int32_t* offsets;  // [E+1]
+  const uint16_t *w1, *w3, *w2;
+  uint16_t* h_perm;  // [cap, I]
+  uint16_t* y_perm;  // [cap, d]
+  // shared experts (S > 0 and all non-null to enable)
+  const uint16_t* x;  // [T, d]
+  const uint16_t *ws1, *ws3, *ws2;
+  uint16_t* h_shared;  // [T, S*I]
+  float* y_shared;     // [T, d]
+};
+// `between` (may be null) is recorded on `st` after the gate/up GEMM is launched.
+cudaError_t launch_grouped_gemms(const Shape& s, const GroupedGemmArgs& a, int num_sms,
+                                 unsigned int* status, uint64_t wait_limit_ns, cudaStream_t st,
+                                 cudaEvent_t between = nullptr);
+
+// ---- combine (combine.cu)
+cudaError_t launch_combine(const Shape& s, const uint16_t* y_perm, const int32_t* row_of,
+                           const float* topk_w, const float* y_shared, uint16_t* y,
+                           cudaStream_t st);
+
+}  // namespace moe

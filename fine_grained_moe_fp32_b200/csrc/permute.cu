@@ -1,0 +1,186 @@
+// Permutation of the (token, slot) pairs into per-expert segments padded to
+// `align` rows (dots.llm1 Technical Report, Method, systems paragraph: expert
+// segments are padded to MMA tile multiples).  A stable counting sort:
+//
+//   permute_count_kernel    per chunk of 256 tokens: expert histogram
+//   permute_scan_kernel     one CTA: per-expert exclusive scan over chunks,
+//                           counts, padded segment offsets, -1 on padding rows
+//   permute_scatter_kernel  per chunk: rank of each pair among the chunk's
+//                           earlier tokens of the same expert (warp ballot
+//                           masks + per-warp prefix), row_of / token_of_row
+//   permute_gather_kernel   one warp per row: x_perm[r] = x[token_of_row[r]]
+//                           (zero for padding rows), 16-byte vectors
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kChunk = kChunkTokens;  // tokens per chunk = threads per CTA
+constexpr int kMaxE = 128;
+constexpr int kWarps = kChunk / 32;
+
+__device__ __forceinline__ void set_status(unsigned int* status, unsigned int code) {
+  if (status != nullptr) atomicCAS(status, 0u, code);
+}
+
+__global__ void __launch_bounds__(kChunk)
+permute_count_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
+                     int32_t* __restrict__ chunk_counts, unsigned int* status) {
+  __shared__ int hist[kMaxE];
+  const int c = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int t = c * kChunk + threadIdx.x;
+  if (t < T) {
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      bool dup = false;
+      for (int jj = 0; jj < j; ++jj) dup |= idx[(size_t)t * k + jj] == e;
+      if (e >= 0 && e < E && !dup)
+        atomicAdd(&hist[e], 1);
+      else
+        set_status(status, DEV_BAD_EXPERT_ID);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_counts[(size_t)c * E + e] = hist[e];
+}
+
+__global__ void __launch_bounds__(kMaxE)
+permute_scan_kernel(const int32_t* __restrict__ chunk_counts, int nchunks, int E, int align,
+                    int64_t cap, int32_t* __restrict__ chunk_base, int32_t* __restrict__ counts,
+                    int32_t* __restrict__ offsets, int32_t* __restrict__ token_of_row) {
+  __shared__ int scan[kMaxE];
+  const int e = threadIdx.x;
+  int total = 0;
+  if (e < E) {
+    for (int c = 0; c < nchunks; ++c) {
+      chunk_base[(size_t)c * E + e] = total;
+      total += chunk_counts[(size_t)c * E + e];
+    }
+    counts[e] = total;
+  }
+  const int padded = e < E ? (int)round_up(total, align) : 0;
+  scan[e] = padded;
+  __syncthreads();
+  // inclusive Hillis-Steele scan over the (at most 128) experts
+  for (int o = 1; o < kMaxE; o <<= 1) {
+    const int v = e >= o ? scan[e - o] : 0;
+    __syncthreads();
+    scan[e] += v;
+    __syncthreads();
+  }
+  const int end = scan[e];
+  const int start = end - padded;
+  if (e < E) {
+    offsets[e] = start;
+    if (e == E - 1) offsets[E] = end;
+    for (int r = start + total; r < end; ++r) token_of_row[r] = -1;
+  }
+  const int used = scan[E - 1];
+  for (int64_t r = used + e; r < cap; r += blockDim.x) token_of_row[r] = -1;
+}
+
+__global__ void __launch_bounds__(kChunk)
+permute_scatter_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
+                       const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ offsets,
+                       int32_t* __restrict__ row_of, int32_t* __restrict__ token_of_row) {
+  __shared__ unsigned int masks[kWarps][kMaxE];
+  __shared__ int pre[kWarps][kMaxE];
+  __shared__ int base[kMaxE];
+  const int c = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kWarps * kMaxE; i += blockDim.x) (&masks[0][0])[i] = 0u;
+  __syncthreads();
+  const int t = c * kChunk + threadIdx.x;
+  const bool tok_ok = t < T;
+  if (tok_ok) {
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      bool dup = false;
+      for (int jj = 0; jj < j; ++jj) dup |= idx[(size_t)t * k + jj] == e;
+      if (e >= 0 && e < E && !dup) atomicOr(&masks[warp][e], 1u << lane);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      pre[w][e] = run;
+      run += __popc(masks[w][e]);
+    }
+    base[e] = offsets[e] + chunk_base[(size_t)c * E + e];
+  }
+  __syncthreads();
+  if (tok_ok) {
+    const unsigned int lt = (1u << lane) - 1u;
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      bool dup = false;
+      for (int jj = 0; jj < j; ++jj) dup |= idx[(size_t)t * k + jj] == e;
+      int row = -1;
+      if (e >= 0 && e < E && !dup) {
+        row = base[e] + pre[warp][e] + __popc(masks[warp][e] & lt);
+        token_of_row[row] = t;
+      }
+      row_of[(size_t)t * k + j] = row;
+    }
+  }
+}
+
+constexpr int kGatherWarps = 8;
+
+__global__ void __launch_bounds__(kGatherWarps * 32)
+permute_gather_kernel(const uint16_t* __restrict__ x, int T, int d,
+                      const int32_t* __restrict__ offsets,
+                      int E, const int32_t* __restrict__ token_of_row, int64_t cap,
+                      uint16_t* __restrict__ x_perm) {
+  const int64_t r = (int64_t)blockIdx.x * kGatherWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= cap || r >= offsets[E]) return;
+  const int tok = token_of_row[r];
+  uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)r * d);
+  const int nv = d / 8;
+  if (tok >= 0 && tok < T) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)tok * d);
+    for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
+  } else {
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    for (int v = lane; v < nv; v += 32) dst[v] = z;
+  }
+}
+
+}  // namespace
+
+size_t permute_scratch_bytes(const Shape& s) {
+  const size_t nchunks = (size_t)ceil_div(s.T, kChunk);
+  return 2 * nchunks * (size_t)s.E * sizeof(int32_t);
+}
+
+cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16_t* x,
+                           int32_t* counts, int32_t* offsets, int32_t* row_of,
+                           int32_t* token_of_row, uint16_t* x_perm, void* scratch,
+                           unsigned int* status, cudaStream_t st) {
+  const int nchunks = (int)ceil_div(s.T, kChunk);
+  int32_t* chunk_counts = static_cast<int32_t*>(scratch);
+  int32_t* chunk_base = chunk_counts + (size_t)nchunks * s.E;
+  if (nchunks > 0) {
+    permute_count_kernel<<<nchunks, kChunk, 0, st>>>(topk_idx, s.T, s.k, s.E, chunk_counts,
+                                                     status);
+  }
+  permute_scan_kernel<<<1, kMaxE, 0, st>>>(chunk_counts, nchunks, s.E, s.align, s.cap,
+                                           chunk_base, counts, offsets, token_of_row);
+  if (nchunks > 0) {
+    permute_scatter_kernel<<<nchunks, kChunk, 0, st>>>(topk_idx, s.T, s.k, s.E, chunk_base,
+                                                       offsets, row_of, token_of_row);
+  }
+  if (s.cap > 0 && x_perm != nullptr) {
+    const unsigned blocks = (unsigned)ceil_div(s.cap, kGatherWarps);
+    permute_gather_kernel<<<blocks, kGatherWarps * 32, 0, st>>>(x, s.T, s.d, offsets, s.E,
+                                                                token_of_row, s.cap, x_perm);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace moe

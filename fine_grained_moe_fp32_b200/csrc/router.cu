@@ -1,0 +1,257 @@
+// Router: FP32 gate GEMM on CUDA cores, then softmax and bias-adjusted top-k
+// per token (dots.llm1 Technical Report, Method: the gate projection runs in
+// FP32 for stable routing; selection uses the auxiliary-loss-free bias).
+//
+// router_gemm_kernel  split-K fp32 GEMM: partial[s, t, e] = sum over the s-th
+//                     k-chunk of x[t, i] * w_gate[e, i]  (x bf16 -> fp32 exactly)
+// router_topk_kernel  one warp per token: z = sum_s partial[s] (s ascending),
+//                     p = softmax(z), key = p + bias, k rounds of warp arg-max
+//                     (equal keys: lower expert id), w = p_sel / sum p_sel
+#include <cuda_bf16.h>
+
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int BT = kRouterBT;  // tokens per tile
+constexpr int BE = 128;        // experts per tile (all of them; E <= 128)
+constexpr int BK = kRouterBK;  // k-chunk in shared memory
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {
+  return __uint_as_float(bits16 << 16);
+}
+
+// 256 threads as a 16 x 16 grid; thread (ty, tx) owns tokens
+// {ty*4 .. ty*4+3, 64+ty*4 .. 64+ty*4+3} and experts {tx*4 .., 64+tx*4 ..}.
+__global__ void __launch_bounds__(kThreads, 2)
+router_gemm_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wg,
+                   float* __restrict__ part, int T, int d, int E, int kchunk) {
+  __shared__ __align__(16) float xs[2][BK][BT];
+  __shared__ __align__(16) float ws[2][BK][BE];
+
+  const int tid = threadIdx.x;
+  const int t0 = blockIdx.x * BT;
+  const int split = blockIdx.y;
+  const int k_begin = split * kchunk;
+  const int k_end = min(d, k_begin + kchunk);
+  const int nk = (k_end - k_begin) / BK;
+
+  // loader roles: one 16-byte bf16 vector of x and two float4 of w_gate per chunk
+  const int lrow = tid & 127;
+  const int lq = tid >> 7;  // 0 or 1
+  const bool x_ok = (t0 + lrow) < T;
+  const bool w_ok = lrow < E;
+  const uint16_t* xrow = x + (size_t)(x_ok ? t0 + lrow : 0) * d;
+  const float* wrow = wg + (size_t)(w_ok ? lrow : 0) * d;
+
+  uint4 xv = make_uint4(0, 0, 0, 0);
+  float4 wv0 = make_float4(0.f, 0.f, 0.f, 0.f), wv1 = wv0;
+  auto gload = [&](int kc) {
+    const int k = k_begin + kc * BK;
+    if (x_ok) xv = *reinterpret_cast<const uint4*>(xrow + k + lq * 8);
+    if (w_ok) {
+      wv0 = *reinterpret_cast<const float4*>(wrow + k + lq * 4);
+      wv1 = *reinterpret_cast<const float4*>(wrow + k + 8 + lq * 4);
+    }
+  };
+  auto sstore = [&](int buf) {
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      xs[buf][lq * 8 + 2 * i][lrow] = bf16_bits_to_float(xw[i] & 0xFFFFu);
+      xs[buf][lq * 8 + 2 * i + 1][lrow] = bf16_bits_to_float(xw[i] >> 16);
+    }
+    ws[buf][lq * 4 + 0][lrow] = wv0.x;
+    ws[buf][lq * 4 + 1][lrow] = wv0.y;
+    ws[buf][lq * 4 + 2][lrow] = wv0.z;
+    ws[buf][lq * 4 + 3][lrow] = wv0.w;
+    ws[buf][8 + lq * 4 + 0][lrow] = wv1.x;
+    ws[buf][8 + lq * 4 + 1][lrow] = wv1.y;
+    ws[buf][8 + lq * 4 + 2][lrow] = wv1.z;
+    ws[buf][8 + lq * 4 + 3][lrow] = wv1.w;
+  };
+
+  const int ty = tid >> 4, tx = tid & 15;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+  if (nk > 0) {
+    gload(0);
+    sstore(0);
+  }
+  __syncthreads();
+  for (int kc = 0; kc < nk; ++kc) {
+    const int buf = kc & 1;
+    if (kc + 1 < nk) gload(kc + 1);
+#pragma unroll
+    for (int kk = 0; kk < BK; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&xs[buf][kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&ws[buf][kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&ws[buf][kk][64 + tx * 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    if (kc + 1 < nk) sstore(buf ^ 1);
+    __syncthreads();
+  }
+
+  float* out = part + (size_t)split * T * E;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int t = t0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
+    if (t >= T) continue;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int e0 = half * 64 + tx * 4;
+      float* dst = out + (size_t)t * E + e0;
+      if (e0 + 3 < E && (E & 3) == 0) {
+        *reinterpret_cast<float4*>(dst) = make_float4(acc[i][half * 4 + 0], acc[i][half * 4 + 1],
+                                                      acc[i][half * 4 + 2], acc[i][half * 4 + 3]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (e0 + j < E) dst[j] = acc[i][half * 4 + j];
+      }
+    }
+  }
+}
+
+struct Cand {
+  float key;
+  int e;
+  float p;
+};
+
+__device__ __forceinline__ bool better(const Cand& a, const Cand& b) {
+  return a.key > b.key || (a.key == b.key && a.e < b.e);
+}
+
+constexpr int kTopkWarps = 8;
+
+__global__ void __launch_bounds__(kTopkWarps * 32)
+router_topk_kernel(const float* __restrict__ part, int splits, const float* __restrict__ bias,
+                   float* __restrict__ probs, int32_t* __restrict__ topk_idx,
+                   float* __restrict__ topk_w, int T, int E, int k) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kTopkWarps + (threadIdx.x >> 5);
+  if (t >= T) return;
+
+  float z[4];
+  bool valid[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = lane + 32 * i;
+    valid[i] = e < E;
+    float s = 0.f;
+    if (valid[i]) {
+      for (int sp = 0; sp < splits; ++sp) s += part[((size_t)sp * T + t) * E + e];
+    }
+    z[i] = valid[i] ? s : -INFINITY;
+  }
+  float m = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float ex[4];
+  float lsum = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    ex[i] = valid[i] ? expf(z[i] - m) : 0.f;
+    lsum += ex[i];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+
+  Cand c[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = lane + 32 * i;
+    const float p = ex[i] / lsum;
+    if (valid[i] && probs != nullptr) probs[(size_t)t * E + e] = p;
+    float key = p + (bias != nullptr && valid[i] ? bias[e] : 0.f);
+    if (!valid[i] || key != key) key = -INFINITY;  // NaN keys rank last
+    c[i].key = key;
+    c[i].e = valid[i] ? e : 0x7fffffff;
+    c[i].p = p;
+  }
+
+  unsigned taken = 0;
+  int my_idx = 0;
+  float my_p = 0.f;
+  for (int r = 0; r < k; ++r) {
+    Cand best = {-INFINITY, 0x7fffffff, 0.f};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (!(taken & (1u << i)) && better(c[i], best)) best = c[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      Cand other;
+      other.key = __shfl_xor_sync(0xffffffffu, best.key, o);
+      other.e = __shfl_xor_sync(0xffffffffu, best.e, o);
+      other.p = __shfl_xor_sync(0xffffffffu, best.p, o);
+      if (better(other, best)) best = other;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (c[i].e == best.e) taken |= 1u << i;
+    if (lane == r) {
+      my_idx = best.e;
+      my_p = best.p;
+    }
+  }
+  float psum = 0.f;
+  for (int r = 0; r < k; ++r) psum += __shfl_sync(0xffffffffu, my_p, r);
+  if (lane < k) {
+    topk_idx[(size_t)t * k + lane] = my_idx;
+    topk_w[(size_t)t * k + lane] = my_p / psum;
+  }
+}
+
+struct SplitPlan {
+  int splits;
+  int kchunk;
+};
+
+SplitPlan plan_splits(const Shape& s, int num_sms) {
+  const int tiles = (int)ceil_div(s.T, BT);
+  const int max_splits = s.d / (BK * 4) > 0 ? s.d / (BK * 4) : 1;
+  int splits = tiles > 0 ? (2 * num_sms) / tiles : 1;
+  if (splits < 1) splits = 1;
+  if (splits > max_splits) splits = max_splits;
+  const int kchunk = (int)round_up(ceil_div(s.d, splits), BK);
+  splits = (int)ceil_div(s.d, kchunk);
+  return {splits, kchunk};
+}
+
+}  // namespace
+
+int router_splits(const Shape& s, int num_sms) { return plan_splits(s, num_sms).splits; }
+
+size_t router_partials_bytes(const Shape& s, int num_sms) {
+  return (size_t)plan_splits(s, num_sms).splits * (size_t)s.T * (size_t)s.E * sizeof(float);
+}
+
+cudaError_t launch_router(const Shape& s, const uint16_t* x, const float* w_gate,
+                          const float* bias, float* probs, int32_t* topk_idx, float* topk_w,
+                          float* partials, int num_sms, cudaStream_t st) {
+  if (s.T == 0) return cudaSuccess;
+  const SplitPlan sp = plan_splits(s, num_sms);
+  dim3 grid((unsigned)ceil_div(s.T, BT), (unsigned)sp.splits);
+  router_gemm_kernel<<<grid, kThreads, 0, st>>>(x, w_gate, partials, s.T, s.d, s.E, sp.kchunk);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  router_topk_kernel<<<(unsigned)ceil_div(s.T, kTopkWarps), kTopkWarps * 32, 0, st>>>(
+      partials, sp.splits, bias, probs, topk_idx, topk_w, s.T, s.E, s.k);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

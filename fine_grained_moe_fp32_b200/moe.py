@@ -1,0 +1,320 @@
+"""ctypes binding of libmoe_b200.so (the C ABI in include/moe_b200.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  torch tensors are used for device memory and the current stream.
+There is no CPU fallback: if the library is missing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_UNSUPPORTED_SHAPE = -2
+MOE_ERR_WORKSPACE = -3
+MOE_ERR_CUDA = -4
+MOE_ERR_TIMEOUT = -5
+
+# every symbol declared in include/moe_b200.h
+EXPORTED = (
+    "moe_capacity", "moe_status_string", "moe_route_workspace_size", "moe_route",
+    "moe_permute_workspace_size", "moe_permute", "moe_grouped_swiglu", "moe_combine",
+    "moe_workspace_size", "moe_forward_layout", "moe_forward", "moe_get_last_device_status",
+    "moe_set_wait_limit_ns", "moe_set_phase_events",
+)
+
+
+class MoeDims(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int), ("d", ctypes.c_int), ("E", ctypes.c_int),
+                ("k", ctypes.c_int), ("I", ctypes.c_int), ("n_shared", ctypes.c_int),
+                ("align", ctypes.c_int)]
+
+
+class MoeWsLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in (
+        "route_partials", "probs", "topk_idx", "topk_w", "counts", "offsets", "row_of",
+        "token_of_row", "permute_scratch", "x_perm", "h_perm", "y_perm", "h_shared",
+        "y_shared", "total")]
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m fine_grained_moe_fp32_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, Z, V = ctypes.POINTER(MoeDims), ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+    sig = {
+        "moe_capacity": (ctypes.c_int64, [P]),
+        "moe_status_string": (ctypes.c_char_p, [I]),
+        "moe_route_workspace_size": (Z, [P]),
+        "moe_route": (I, [P, V, V, V, V, V, V, V, Z, V]),
+        "moe_permute_workspace_size": (Z, [P]),
+        "moe_permute": (I, [P, V, V, V, V, V, V, V, V, Z, V]),
+        "moe_grouped_swiglu": (I, [P, V, V, V, V, V, V, V, V]),
+        "moe_combine": (I, [P, V, V, V, V, V, V]),
+        "moe_workspace_size": (Z, [P]),
+        "moe_forward_layout": (I, [P, ctypes.POINTER(MoeWsLayout)]),
+        "moe_forward": (I, [P, V, V, V, V, V, V, V, V, V, V, V, Z, V]),
+        "moe_get_last_device_status": (I, [V]),
+        "moe_set_wait_limit_ns": (I, [ctypes.c_uint64]),
+        "moe_set_phase_events": (I, [ctypes.POINTER(ctypes.c_void_p), I]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return load().moe_status_string(status).decode()
+    except RuntimeError:
+        return "unknown"
+
+
+def _check(rc: int, what: str):
+    if rc != MOE_OK:
+        raise MoEError(rc, what)
+
+
+def dims(T, d, E, k, I, n_shared, align=16) -> MoeDims:
+    return MoeDims(int(T), int(d), int(E), int(k), int(I), int(n_shared), int(align))
+
+
+def dims_of(cfg, T=None, align=16) -> MoeDims:
+    return dims(cfg.T if T is None else T, cfg.d, cfg.E, cfg.k, cfg.I, cfg.S, align)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors passed to the library must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the library must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _expect(t, dtype, shape, name):
+    if t is None:
+        return
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected {dtype} {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
+def capacity(dm: MoeDims) -> int:
+    return int(load().moe_capacity(ctypes.byref(dm)))
+
+
+def workspace_size(dm: MoeDims) -> int:
+    return int(load().moe_workspace_size(ctypes.byref(dm)))
+
+
+def route_workspace_size(dm: MoeDims) -> int:
+    return int(load().moe_route_workspace_size(ctypes.byref(dm)))
+
+
+def permute_workspace_size(dm: MoeDims) -> int:
+    return int(load().moe_permute_workspace_size(ctypes.byref(dm)))
+
+
+def forward_layout(dm: MoeDims) -> dict:
+    L = MoeWsLayout()
+    _check(load().moe_forward_layout(ctypes.byref(dm), ctypes.byref(L)), "moe_forward_layout")
+    return {n: getattr(L, n) for n, _ in MoeWsLayout._fields_}
+
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A uint8 device buffer of at least nbytes (torch's allocator aligns to 512 B)."""
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------------ calls
+
+def route(dm, x, w_gate, bias, probs, topk_idx, topk_w, workspace, stream=None):
+    _expect(x, torch.bfloat16, (dm.T, dm.d), "x")
+    _expect(w_gate, torch.float32, (dm.E, dm.d), "w_gate")
+    _expect(bias, torch.float32, (dm.E,), "bias")
+    _expect(probs, torch.float32, (dm.T, dm.E), "probs")
+    _expect(topk_idx, torch.int32, (dm.T, dm.k), "topk_idx")
+    _expect(topk_w, torch.float32, (dm.T, dm.k), "topk_w")
+    rc = load().moe_route(ctypes.byref(dm), _ptr(x), _ptr(w_gate), _ptr(bias), _ptr(probs),
+                          _ptr(topk_idx), _ptr(topk_w), _ptr(workspace),
+                          workspace.numel() if workspace is not None else 0, _stream(stream))
+    _check(rc, "moe_route")
+
+
+def permute(dm, topk_idx, x, counts, offsets, row_of, token_of_row, x_perm, workspace,
+            stream=None):
+    cap = capacity(dm)
+    _expect(topk_idx, torch.int32, (dm.T, dm.k), "topk_idx")
+    _expect(x, torch.bfloat16, (dm.T, dm.d), "x")
+    _expect(counts, torch.int32, (dm.E,), "counts")
+    _expect(offsets, torch.int32, (dm.E + 1,), "offsets")
+    _expect(row_of, torch.int32, (dm.T * dm.k,), "row_of")
+    _expect(token_of_row, torch.int32, (cap,), "token_of_row")
+    _expect(x_perm, torch.bfloat16, (cap, dm.d), "x_perm")
+    rc = load().moe_permute(ctypes.byref(dm), _ptr(topk_idx), _ptr(x), _ptr(counts),
+                            _ptr(offsets), _ptr(row_of), _ptr(token_of_row), _ptr(x_perm),
+                            _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                            _stream(stream))
+    _check(rc, "moe_permute")
+
+
+def grouped_swiglu(dm, x_perm, offsets, w1, w3, w2, h_perm, y_perm, stream=None):
+    cap = capacity(dm)
+    _expect(x_perm, torch.bfloat16, (cap, dm.d), "x_perm")
+    _expect(offsets, torch.int32, (dm.E + 1,), "offsets")
+    _expect(w1, torch.bfloat16, (dm.E, dm.I, dm.d), "w1")
+    _expect(w3, torch.bfloat16, (dm.E, dm.I, dm.d), "w3")
+    _expect(w2, torch.bfloat16, (dm.E, dm.d, dm.I), "w2")
+    _expect(h_perm, torch.bfloat16, (cap, dm.I), "h_perm")
+    _expect(y_perm, torch.bfloat16, (cap, dm.d), "y_perm")
+    rc = load().moe_grouped_swiglu(ctypes.byref(dm), _ptr(x_perm), _ptr(offsets), _ptr(w1),
+                                   _ptr(w3), _ptr(w2), _ptr(h_perm), _ptr(y_perm),
+                                   _stream(stream))
+    _check(rc, "moe_grouped_swiglu")
+
+
+def combine(dm, y_perm, row_of, topk_w, y_shared, y, stream=None):
+    cap = capacity(dm)
+    _expect(y_perm, torch.bfloat16, (cap, dm.d), "y_perm")
+    _expect(row_of, torch.int32, (dm.T * dm.k,), "row_of")
+    _expect(topk_w, torch.float32, (dm.T, dm.k), "topk_w")
+    _expect(y_shared, torch.float32, (dm.T, dm.d), "y_shared")
+    _expect(y, torch.bfloat16, (dm.T, dm.d), "y")
+    rc = load().moe_combine(ctypes.byref(dm), _ptr(y_perm), _ptr(row_of), _ptr(topk_w),
+                            _ptr(y_shared), _ptr(y), _stream(stream))
+    _check(rc, "moe_combine")
+
+
+def forward(dm, x, w_gate, bias, w1, w3, w2, ws1, ws3, ws2, y, workspace, stream=None):
+    _expect(x, torch.bfloat16, (dm.T, dm.d), "x")
+    _expect(w_gate, torch.float32, (dm.E, dm.d), "w_gate")
+    _expect(bias, torch.float32, (dm.E,), "bias")
+    _expect(w1, torch.bfloat16, (dm.E, dm.I, dm.d), "w1")
+    _expect(w3, torch.bfloat16, (dm.E, dm.I, dm.d), "w3")
+    _expect(w2, torch.bfloat16, (dm.E, dm.d, dm.I), "w2")
+    if dm.n_shared > 0:
+        _expect(ws1, torch.bfloat16, (dm.n_shared, dm.I, dm.d), "ws1")
+        _expect(ws3, torch.bfloat16, (dm.n_shared, dm.I, dm.d), "ws3")
+        _expect(ws2, torch.bfloat16, (dm.n_shared, dm.d, dm.I), "ws2")
+    _expect(y, torch.bfloat16, (dm.T, dm.d), "y")
+    rc = load().moe_forward(ctypes.byref(dm), _ptr(x), _ptr(w_gate), _ptr(bias), _ptr(w1),
+                            _ptr(w3), _ptr(w2), _ptr(ws1), _ptr(ws3), _ptr(ws2), _ptr(y),
+                            _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "moe_forward")
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream; return and clear the device status word."""
+    return int(load().moe_get_last_device_status(_stream(stream)))
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    load().moe_set_wait_limit_ns(int(ns))
+
+
+PHASES = ("router", "permute", "gemm_gate_up_swiglu", "gemm_down", "combine")
+
+
+def set_phase_events(events) -> None:
+    """Record torch.cuda.Event objects between the kernels of moe_forward
+    (6 events: before the router, then after each of the 5 phases); None
+    turns the hook off."""
+    if events is None:
+        _check(load().moe_set_phase_events(None, 0), "moe_set_phase_events")
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(load().moe_set_phase_events(arr, len(events)), "moe_set_phase_events")
+
+
+# ------------------------------------------------------------------ helpers
+
+def workspace_views(dm: MoeDims, ws: torch.Tensor) -> dict:
+    """Typed views of the intermediates moe_forward leaves in its workspace."""
+    L = forward_layout(dm)
+    cap = capacity(dm)
+    T, d, E, k, I, S = dm.T, dm.d, dm.E, dm.k, dm.I, dm.n_shared
+
+    def view(off, n, dtype, shape):
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        return ws[off:off + nbytes].view(dtype).view(*shape)
+
+    return {
+        "probs": view(L["probs"], T * E, torch.float32, (T, E)),
+        "topk_idx": view(L["topk_idx"], T * k, torch.int32, (T, k)),
+        "topk_w": view(L["topk_w"], T * k, torch.float32, (T, k)),
+        "counts": view(L["counts"], E, torch.int32, (E,)),
+        "offsets": view(L["offsets"], E + 1, torch.int32, (E + 1,)),
+        "row_of": view(L["row_of"], T * k, torch.int32, (T * k,)),
+        "token_of_row": view(L["token_of_row"], cap, torch.int32, (cap,)),
+        "x_perm": view(L["x_perm"], cap * d, torch.bfloat16, (cap, d)),
+        "h_perm": view(L["h_perm"], cap * I, torch.bfloat16, (cap, I)),
+        "y_perm": view(L["y_perm"], cap * d, torch.bfloat16, (cap, d)),
+        "h_shared": view(L["h_shared"], T * S * I, torch.bfloat16, (T, S * I)),
+        "y_shared": view(L["y_shared"], T * d, torch.float32, (T, d)),
+    }
+
+
+class MoELayer:
+    """The layer with its weights resident on one device; ``__call__`` runs
+    moe_forward into a reusable workspace."""
+
+    def __init__(self, inputs: dict, align: int = 16, device="cuda"):
+        cfg = inputs["cfg"]
+        self.cfg = cfg
+        self.align = align
+        self.device = torch.device(device)
+        to = lambda t: t.to(self.device).contiguous()  # noqa: E731
+        self.w_gate = to(inputs["w_gate"])
+        self.bias = to(inputs["bias"])
+        self.w1, self.w3, self.w2 = to(inputs["w1"]), to(inputs["w3"]), to(inputs["w2"])
+        self.ws1, self.ws3, self.ws2 = to(inputs["ws1"]), to(inputs["ws3"]), to(inputs["ws2"])
+        self._ws = None
+        self._ws_T = -1
+
+    def dims(self, T: int) -> MoeDims:
+        c = self.cfg
+        return dims(T, c.d, c.E, c.k, c.I, c.S, self.align)
+
+    def workspace(self, T: int) -> torch.Tensor:
+        if self._ws is None or self._ws_T != T:
+            self._ws = alloc_workspace(workspace_size(self.dims(T)), self.device)
+            self._ws_T = T
+        return self._ws
+
+    def __call__(self, x: torch.Tensor, y: torch.Tensor | None = None, stream=None):
+        T = x.shape[0]
+        dm = self.dims(T)
+        if y is None:
+            y = torch.empty((T, self.cfg.d), dtype=torch.bfloat16, device=self.device)
+        forward(dm, x, self.w_gate, self.bias, self.w1, self.w3, self.w2, self.ws1, self.ws3,
+                self.ws2, y, self.workspace(T), stream)
+        return y

@@ -1,0 +1,232 @@
+/*
+ * moe_b200.h -- C ABI of the dots.llm1 fine-grained MoE FFN layer for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The layer (dots.llm1 Technical Report, Method; "Model Architecture Features"
+ * on the kdjingpai.com page): an FP32 gate scores E = 128 routed experts, the
+ * auxiliary-loss-free per-expert bias picks the top k = 6, two shared experts
+ * are always on, every expert is a SwiGLU feed-forward network, and the
+ * outputs are summed with the renormalised gate weights.  The grouped GEMM
+ * pads every expert's token segment to a multiple of the MMA tile (Technical
+ * Report, Key claims / Method, systems paragraph).
+ *
+ * Conventions shared by every call
+ * ---------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    never allocates device memory; scratch ("workspace") is caller-provided
+ *    and its size is queried first.
+ *  - Layouts are row-major.  Weights follow the [out, in] convention:
+ *      w1, w3 [E, I, d]  gate / up projections of routed expert e
+ *      w2     [E, d, I]  down projection of routed expert e
+ *      ws1, ws3 [S, I, d], ws2 [S, d, I]  the S shared experts (same I)
+ *  - bf16 tensors are passed as moe_bf16 (the raw 16-bit pattern).
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and does no host synchronisation.  Argument errors are
+ *    detected on the host before anything is launched and are returned as a
+ *    negative status.  Errors that only the device can see (an expert id out
+ *    of range, a bounded wait that ran out) are recorded in a per-device
+ *    status word that moe_get_last_device_status() returns.
+ *  - Routing convention (readings where the pages are silent): softmax over
+ *    the E fp32 logits; the bias is added to the probabilities for the
+ *    selection only; the chosen probabilities are renormalised to sum to 1;
+ *    equal keys rank the lower expert id first; shared experts have weight 1;
+ *    SwiGLU h = silu(w1 x) * (w3 x), silu(g) = g / (1 + exp(-g)).
+ *  - Shape limits: 1 <= E <= 128, 1 <= k <= min(E, 8), d % 128 == 0,
+ *    I % 64 == 0, align % 16 == 0, 0 <= n_shared <= 4, T >= 0.
+ *    Violations return MOE_ERR_UNSUPPORTED_SHAPE.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16;
+
+/* Status codes. */
+enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,       /* null pointer, negative size, bad idx */
+  MOE_ERR_UNSUPPORTED_SHAPE = -2, /* shape outside the limits above       */
+  MOE_ERR_WORKSPACE = -3,         /* workspace missing, small or unaligned */
+  MOE_ERR_CUDA = -4,              /* a CUDA runtime call failed            */
+  MOE_ERR_TIMEOUT = -5            /* a bounded device-side wait ran out    */
+};
+
+/* Layer dimensions.
+ *   T tokens, d hidden size, E routed experts, k experts chosen per token,
+ *   I intermediate size of every expert (routed and shared), n_shared shared
+ *   experts, align = segment padding granularity in rows (multiple of 16). */
+typedef struct moe_dims {
+  int T, d, E, k, I, n_shared, align;
+} moe_dims;
+
+/* Rows of the permuted buffers: T*k + E*(align-1), the most any routing can
+ * need once every segment is rounded up to `align`.  Returns 0 on bad dims. */
+int64_t moe_capacity(const moe_dims* dims);
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_string(int status);
+
+/* ------------------------------------------------------------------------
+ * moe_route -- the FP32 gate and bias-adjusted top-k selection.
+ * Technical Report, Method: gate projection in FP32, auxiliary-loss-free
+ * bias, top-6 of 128.
+ *
+ *   x        [T, d]  bf16 tokens
+ *   w_gate   [E, d]  fp32 gate weights
+ *   bias     [E]     fp32 selection bias (may be NULL: zero bias)
+ *   probs    [T, E]  fp32 out: softmax of the logits (may be NULL)
+ *   topk_idx [T, k]  int32 out: chosen experts by descending p + bias
+ *   topk_w   [T, k]  fp32 out: renormalised probabilities of the chosen experts
+ *   workspace        device scratch of moe_route_workspace_size() bytes,
+ *                    256-byte aligned (partial gate logits of the split-K
+ *                    fp32 GEMM)
+ * The logits are accumulated in fp32 in a fixed order, so results are
+ * deterministic for given dims.  Returns MOE_OK or a negative status.
+ * ---------------------------------------------------------------------- */
+size_t moe_route_workspace_size(const moe_dims* dims);
+int moe_route(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
+              const float* bias, float* probs, int32_t* topk_idx,
+              float* topk_w, void* workspace, size_t workspace_bytes,
+              void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_permute -- counting sort of the (token, slot) pairs into per-expert
+ * segments padded to `align` rows, and the row gather of x.
+ * Technical Report, Method (systems paragraph): expert segments are padded to
+ * tile multiples so every MMA tile holds rows of one expert only.
+ *
+ *   topk_idx     [T, k]     int32 expert ids (each in [0, E))
+ *   x            [T, d]     bf16 tokens
+ *   counts       [E]        int32 out: pairs routed to each expert
+ *   offsets      [E+1]      int32 out: first row of each segment; segment e
+ *                           spans counts[e] rounded up to `align` rows
+ *   row_of       [T*k]      int32 out: row of pair (t, j) at index t*k + j;
+ *                           rows of a segment follow ascending token id
+ *   token_of_row [cap]      int32 out: token of each row; -1 for padding
+ *                           rows and for rows >= offsets[E]
+ *   x_perm       [cap, d]   bf16 out: x_perm[r] = x[token_of_row[r]], padding
+ *                           rows inside segments are zero; rows at or after
+ *                           offsets[E] are not written
+ *   workspace               moe_permute_workspace_size() bytes (per-chunk
+ *                           expert histograms)
+ * cap = moe_capacity(dims).  Ids out of range are skipped and flagged as
+ * MOE_ERR_INVALID_ARG in the device status word.
+ * ---------------------------------------------------------------------- */
+size_t moe_permute_workspace_size(const moe_dims* dims);
+int moe_permute(const moe_dims* dims, const int32_t* topk_idx,
+                const moe_bf16* x, int32_t* counts, int32_t* offsets,
+                int32_t* row_of, int32_t* token_of_row, moe_bf16* x_perm,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_grouped_swiglu -- the grouped SwiGLU expert GEMMs over the segments.
+ * Technical Report, Key claims / Method (grouped GEMM over tile-padded expert
+ * segments); SwiGLU experts per the Model Architecture Features paragraph.
+ * tcgen05 tensor-core MMAs (bf16 in, fp32 accumulate in tensor memory), fed by
+ * TMA; SwiGLU is fused into the epilogue of the gate/up GEMM.
+ *
+ *   x_perm  [cap, d]   bf16 segment rows (moe_permute output)
+ *   offsets [E+1]      int32 segment starts (moe_permute output)
+ *   w1, w3  [E, I, d]  bf16;  w2 [E, d, I] bf16
+ *   h_perm  [cap, I]   bf16 out: silu(x w1^T) * (x w3^T) for every segment row
+ *   y_perm  [cap, d]   bf16 out: h w2^T for every segment row
+ * Rows outside [0, offsets[E]) are neither read nor written.  Padding rows are
+ * computed like the others (zero rows give zero outputs).  No workspace.
+ * ---------------------------------------------------------------------- */
+int moe_grouped_swiglu(const moe_dims* dims, const moe_bf16* x_perm,
+                       const int32_t* offsets, const moe_bf16* w1,
+                       const moe_bf16* w3, const moe_bf16* w2,
+                       moe_bf16* h_perm, moe_bf16* y_perm, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_combine -- weighted un-permute and shared-expert add.
+ * Technical Report, Method: output = shared experts (weight 1) + the k routed
+ * experts weighted by the gate.
+ *
+ *   y_perm   [cap, d]  bf16 routed expert outputs per segment row
+ *   row_of   [T*k]     int32 row of each (token, slot) pair
+ *   topk_w   [T, k]    fp32 weights
+ *   y_shared [T, d]    fp32 sum of the shared experts' outputs (may be NULL)
+ *   y        [T, d]    bf16 out: y[t] = y_shared[t] + sum_j w[t,j] y_perm[row_of[t*k+j]]
+ * The sum runs in fp32, slot j in ascending order, and is rounded once.
+ * ---------------------------------------------------------------------- */
+int moe_combine(const moe_dims* dims, const moe_bf16* y_perm,
+                const int32_t* row_of, const float* topk_w,
+                const float* y_shared, moe_bf16* y, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_forward -- the whole layer in one call: route, permute, grouped SwiGLU
+ * GEMMs for the routed experts and the shared experts, combine.
+ *
+ *   x [T, d] bf16; w_gate [E, d] fp32; bias [E] fp32 (NULL = zero)
+ *   w1, w3 [E, I, d], w2 [E, d, I] bf16 routed experts
+ *   ws1, ws3 [S, I, d], ws2 [S, d, I] bf16 shared experts (NULL iff S == 0)
+ *   y [T, d] bf16 out
+ *   workspace  moe_workspace_size() bytes, 256-byte aligned.  After the call
+ *              it holds every intermediate at the offsets moe_forward_layout()
+ *              reports (probs, idx, weights, counts, offsets, row_of,
+ *              token_of_row, x_perm, h_perm, y_perm, h_shared, y_shared).
+ * ---------------------------------------------------------------------- */
+typedef struct moe_ws_layout {
+  size_t route_partials;  /* fp32 [splits, T, E] split-K partial logits    */
+  size_t probs;           /* fp32 [T, E]                                   */
+  size_t topk_idx;        /* int32 [T, k]                                  */
+  size_t topk_w;          /* fp32 [T, k]                                   */
+  size_t counts;          /* int32 [E]                                     */
+  size_t offsets;         /* int32 [E+1]                                   */
+  size_t row_of;          /* int32 [T*k]                                   */
+  size_t token_of_row;    /* int32 [cap]                                   */
+  size_t permute_scratch; /* moe_permute_workspace_size() bytes            */
+  size_t x_perm;          /* bf16 [cap, d]                                 */
+  size_t h_perm;          /* bf16 [cap, I]                                 */
+  size_t y_perm;          /* bf16 [cap, d]                                 */
+  size_t h_shared;        /* bf16 [T, S*I]; column s*I + i = shared expert s */
+  size_t y_shared;        /* fp32 [T, d]   sum of the shared experts        */
+  size_t total;           /* = moe_workspace_size()                        */
+} moe_ws_layout;
+
+size_t moe_workspace_size(const moe_dims* dims);
+int moe_forward_layout(const moe_dims* dims, moe_ws_layout* layout);
+int moe_forward(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
+                const float* bias, const moe_bf16* w1, const moe_bf16* w3,
+                const moe_bf16* w2, const moe_bf16* ws1, const moe_bf16* ws3,
+                const moe_bf16* ws2, moe_bf16* y, void* workspace,
+                size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Device status and bounded waits.
+ *
+ * moe_get_last_device_status: synchronises `stream`, returns the first error
+ * the kernels recorded on the current device since the last call (MOE_OK if
+ * none) and clears it.  MOE_ERR_TIMEOUT means a pipeline wait inside a kernel
+ * gave up; the kernel then drained its own copies, freed its tensor memory and
+ * returned, so the context stays usable.
+ *
+ * moe_set_wait_limit_ns: limit of every pipeline wait inside the GEMM kernels
+ * (default 1e9 ns; 0 restores the default).  A test hook: a tiny limit makes
+ * the waits run out on purpose.  Process-wide, not thread-safe.
+ * ---------------------------------------------------------------------- */
+int moe_get_last_device_status(void* stream);
+int moe_set_wait_limit_ns(uint64_t ns);
+
+/* ------------------------------------------------------------------------
+ * moe_set_phase_events -- measurement hook.  With n >= 6 CUDA events
+ * (cudaEvent_t handles owned by the caller), every later moe_forward records
+ * events[0] before its first kernel and events[1..5] after the router, the
+ * permutation, the gate/up GEMM, the down GEMM and the combine, on its stream.
+ * n == 0 (or events == NULL) turns the hook off.  Process-wide; the events
+ * must outlive every moe_forward issued while they are set.
+ * ---------------------------------------------------------------------- */
+int moe_set_phase_events(void* const* events, int n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -49,6 +49,14 @@ def _f64(a) -> np.ndarray:
     return np.asarray(a, dtype=np.float64)
 
 
+def _rows(a, rows) -> np.ndarray:
+    """a[rows] as float64, for a torch tensor or an array."""
+    if hasattr(a, "detach"):
+        import torch
+        return _f64(a[torch.as_tensor(np.asarray(rows), device=a.device)])
+    return _f64(np.asarray(a)[np.asarray(rows)])
+
+
 # --------------------------------------------------------------------------
 # Routing (Technical Report, Method: FP32 gate, aux-loss-free bias, top-6)
 # --------------------------------------------------------------------------
@@ -75,16 +83,18 @@ def select_topk(keys, k: int) -> np.ndarray:
     return order[:, :k].astype(np.int64)
 
 
-def route(x, w_gate, bias, k: int) -> dict:
+def route(x, w_gate, bias, k: int, idx=None) -> dict:
     """Gate, softmax, bias-adjusted top-k selection and renormalised weights.
 
     Returns probs [T,E], keys [T,E] (= probs + bias), idx [T,k] (descending key)
-    and w [T,k] (probs of the chosen experts divided by their sum).
+    and w [T,k] (probs of the chosen experts divided by their sum).  A given
+    ``idx`` replaces the selection (used where two keys tie within rounding and
+    either choice is correct); the weights still follow from the probs.
     """
     z = gate_logits(x, w_gate)
     p = softmax(z)
     keys = p + _f64(bias)[None, :]
-    idx = select_topk(keys, k)
+    idx = select_topk(keys, k) if idx is None else np.asarray(idx, dtype=np.int64)
     p_sel = np.take_along_axis(p, idx, axis=-1)
     w = p_sel / p_sel.sum(axis=-1, keepdims=True)
     return {"logits": z, "probs": p, "keys": keys, "idx": idx, "w": w}
@@ -176,19 +186,19 @@ def swiglu_expert(xr, w1, w3, w2):
 # Whole layer
 # --------------------------------------------------------------------------
 
-def forward(inp: dict, align: int = 16) -> dict:
+def forward(inp: dict, align: int = 16, idx=None) -> dict:
     """The MoE FFN forward in the pages' order: route, permute into padded
     segments, one SwiGLU per segment, shared experts on every token, weighted
     combine back to token order.
 
     ``inp`` holds x, w_gate, bias, w1, w3, w2, ws1, ws3, ws2 (torch or numpy)
-    and the config (for k).
+    and the config (for k).  ``idx`` optionally fixes the selection.
     """
     cfg = inp["cfg"]
     k, E = cfg.k, cfg.E
     x = _f64(inp["x"])
     T = x.shape[0]
-    r = route(x, inp["w_gate"], inp["bias"], k)
+    r = route(x, inp["w_gate"], inp["bias"], k, idx)
     pm = permute(r["idx"], E, align)
     x_perm = gather_rows(x, pm["token_of_row"])
     off = pm["offsets"]
@@ -217,27 +227,24 @@ def forward(inp: dict, align: int = 16) -> dict:
             "y": y}
 
 
-def forward_tokens(inp: dict, tokens) -> dict:
-    """The layer output for a subset of tokens, one token at a time: route the
-    token, run its k chosen experts and the shared experts on it, sum with the
-    weights.  Used for sampled parity at sizes the full oracle cannot run."""
+def forward_tokens(inp: dict, tokens, idx=None) -> dict:
+    """The layer output for a subset of tokens, without the permutation:
+    y_t = sum_s F_s(x_t) + sum_j w_tj F_{e_tj}(x_t), with F_e the SwiGLU expert
+    e.  Each expert is applied to the sampled tokens that chose it.  Used for
+    sampled parity at sizes the full oracle cannot run.  ``idx`` optionally
+    fixes the selection of these tokens."""
     cfg = inp["cfg"]
     tokens = np.asarray(tokens, dtype=np.int64)
-    xt = _f64(inp["x"][tokens])
-    r = route(xt, inp["w_gate"], inp["bias"], cfg.k)
+    xt = _rows(inp["x"], tokens)
+    r = route(xt, inp["w_gate"], inp["bias"], cfg.k, idx)
     ys = np.zeros_like(xt)
-    for n in range(len(tokens)):
-        acc = np.zeros(xt.shape[1])
-        for s in range(inp["ws1"].shape[0]):
-            o, _, _, _ = swiglu_expert(xt[n:n + 1], inp["ws1"][s], inp["ws3"][s],
-                                       inp["ws2"][s])
-            acc += o[0]
-        for j in range(cfg.k):
-            e = int(r["idx"][n, j])
-            o, _, _, _ = swiglu_expert(xt[n:n + 1], inp["w1"][e], inp["w3"][e],
-                                       inp["w2"][e])
-            acc += r["w"][n, j] * o[0]
-        ys[n] = acc
+    for s in range(inp["ws1"].shape[0]):
+        o, _, _, _ = swiglu_expert(xt, inp["ws1"][s], inp["ws3"][s], inp["ws2"][s])
+        ys += o
+    for e in np.unique(r["idx"]):
+        n, j = np.nonzero(r["idx"] == e)
+        o, _, _, _ = swiglu_expert(xt[n], inp["w1"][int(e)], inp["w3"][int(e)], inp["w2"][int(e)])
+        ys[n] += r["w"][n, j][:, None] * o
     return {**r, "tokens": tokens, "y": ys}
 
 

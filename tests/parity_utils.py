@@ -1,0 +1,80 @@
+"""Comparison rules between the CUDA path and the fp64 oracle.
+
+Tolerances (derived from the arithmetic; the layer-output bound is the one the
+workload specification fixes):
+  * routing ids: bit-exact, except where the oracle's fp64 keys of the two
+    choices differ by less than 1e-6 (a tie within rounding; either choice is
+    correct, lower id first is the rule on exact ties);
+  * fp32 router probabilities and weights: relative error <= 1e-5;
+  * integer / index outputs of the permutation: bit-exact, against the oracle
+    run on the GPU's own routing;
+  * bf16 intermediates (h, y_perm): every element within 2^-8 of its own
+    magnitude (one bf16 rounding plus fp32 accumulation) plus 1e-3 rms;
+  * the layer output y (bf16): max |gpu - oracle| <= 2e-2 * rms(oracle).
+"""
+import numpy as np
+import torch
+
+TIE_EPS = 1e-6
+PROB_RTOL = 1e-5
+BF16_REL = 2.0 ** -8
+Y_RMS_FRAC = 2e-2
+
+
+def to_np(t):
+    return t.detach().to("cpu").double().numpy() if torch.is_tensor(t) else np.asarray(t)
+
+
+def rms(a):
+    a = np.asarray(a, dtype=np.float64)
+    return float(np.sqrt(np.mean(a * a))) if a.size else 0.0
+
+
+def check_routing(idx_gpu, keys_ref, idx_ref, k):
+    """Returns the number of tokens decided by a tie; raises on a real mismatch."""
+    idx_gpu = np.asarray(idx_gpu)
+    T = idx_gpu.shape[0]
+    assert idx_gpu.shape == (T, k)
+    assert ((idx_gpu >= 0) & (idx_gpu < keys_ref.shape[1])).all(), "expert id out of range"
+    for t in range(T):
+        assert len(set(idx_gpu[t].tolist())) == k, f"token {t}: repeated expert"
+    bad = np.nonzero((idx_gpu != idx_ref).any(axis=1))[0]
+    for t in bad:
+        kg = keys_ref[t, idx_gpu[t]]
+        kr = keys_ref[t, idx_ref[t]]
+        assert np.all(np.abs(kg - kr) < TIE_EPS), (
+            f"token {t}: gpu {idx_gpu[t].tolist()} oracle {idx_ref[t].tolist()} "
+            f"key gaps {np.abs(kg - kr).tolist()}")
+    return len(bad)
+
+
+def check_probs(p_gpu, p_ref):
+    p_gpu = to_np(p_gpu)
+    err = np.abs(p_gpu - p_ref) / np.maximum(np.abs(p_ref), 1e-30)
+    assert err.max() <= PROB_RTOL, f"probs rel err {err.max():.3e}"
+    return float(err.max())
+
+
+def check_bf16_elementwise(got, ref, what):
+    got, ref = to_np(got), np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    bound = BF16_REL * np.abs(ref) + 1e-3 * rms(ref) + 1e-30
+    err = np.abs(got - ref)
+    worst = np.unravel_index(np.argmax(err / bound), err.shape) if err.size else None
+    assert np.all(err <= bound), (
+        f"{what}: worst at {worst}: got {got[worst]} ref {ref[worst]} bound {bound[worst]}")
+    return float(err.max()) if err.size else 0.0
+
+
+def check_output(y_gpu, y_ref, what="y"):
+    y_gpu, y_ref = to_np(y_gpu), np.asarray(y_ref, dtype=np.float64)
+    assert np.isfinite(y_gpu).all(), f"{what}: non-finite values"
+    r = rms(y_ref)
+    err = float(np.abs(y_gpu - y_ref).max()) if y_ref.size else 0.0
+    assert err <= Y_RMS_FRAC * r + 1e-30, f"{what}: max err {err:.4e} > {Y_RMS_FRAC} * rms {r:.4e}"
+    return err / r if r > 0 else 0.0
+
+
+def np_inputs(inp):
+    """Oracle view of a workload (tensors stay torch; the oracle converts)."""
+    return {k: (v.detach().cpu() if torch.is_tensor(v) else v) for k, v in inp.items()}
