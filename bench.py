@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""Benchmark of the dots.llm1 MoE FFN layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
+
+One step = one moe_forward (router, permutation, grouped SwiGLU GEMMs with the
+shared experts, combine) over one batch of T synthetic tokens.  The default
+workload is the decode-sized layer (T=128, d=5120, 128 experts top-6 + 2
+shared, I=1408), whose throughput is bound by streaming the expert weights
+from HBM.  Under torchrun every rank runs its own batch with replicated
+weights and no collective on the data path (data-parallel replicas, weak
+scaling); the timed region is bracketed by a barrier and synchronisation on
+both sides and the time is the max over ranks.
+
+Prints ONE JSON line on rank 0.  `--impl reference` times the fp64 CPU oracle
+on host cores on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from fine_grained_moe_fp32_b200.workloads import CONFIGS, make_inputs  # noqa: E402
+
+METRIC = "MoE-layer tokens/s (bf16, d=5120, 128E top-6 + 2 shared) and % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = 9  # router gemm + top-k, 4 permutation kernels, 2 grouped GEMMs, combine
+
+
+# ---------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+GEMM_SOURCES = ("fine_grained_moe_fp32_b200/csrc/grouped_gemm.cu",
+                "fine_grained_moe_fp32_b200/csrc/ptx_sm100.cuh")
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel: str, workload: str):
+    """dram read+write bytes per launch from a committed ncu summary
+    (profiles/<kernel>__<workload>.txt: 'traffic_bytes_per_launch: N' and the
+    'kernel_source_hash' of the kernel it was captured on).  None when there
+    is no capture or the kernel has changed since."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}__{workload}.txt")
+    fields = {}
+    try:
+        with open(path) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    fields[k.strip()] = v.strip()
+    except OSError:
+        return None
+    if fields.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    try:
+        return float(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons of one GPU, sampled in the
+    background while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int, interval_ms: int = 50):
+        self.rows = []
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", str(interval_ms)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, RuntimeError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [c.strip() for c in line.split(",")]))
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = [r for t, r in self.rows if t0 - 0.06 <= t <= t1 + 0.06] or [r for _, r in self.rows]
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[0]))
+                smax.append(float(r[1]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[4:8]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world: int, T: int, steps: int, ms_max: float) -> float:
+    """Tokens per second of the whole job: every rank's tokens over the
+    slowest rank's time."""
+    return world * T * steps / (ms_max / 1e3)
+
+
+def shard_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own token batch; the weights are replicated."""
+    return seed + 7919 * rank
+
+
+def gemm_units(cfg, T, counts):
+    """Algorithmic work of the two grouped GEMMs for one step (padding not
+    counted): bytes that must move and flops that must be done."""
+    d, I, S, k = cfg.d, cfg.I, cfg.S, cfg.k
+    touched = int((counts > 0).sum())
+    rows = T * k
+    g1_bytes = (touched + S) * 2 * I * d * 2 + (rows + T) * d * 2 + (rows + T * S) * I * 2
+    g2_bytes = (touched + S) * d * I * 2 + (rows + T * S) * I * 2 + rows * d * 2 + T * d * 4
+    g1_flops = 2 * (rows * 2 * I + T * 2 * S * I) * d
+    g2_flops = 2 * (rows * I + T * S * I) * d
+    return {"touched_experts": touched, "gemm_gate_up_swiglu": (g1_bytes, g1_flops),
+            "gemm_down": (g2_bytes, g2_flops)}
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 0) for i in threadpool_info()), default=0)
+        if n:
+            return n
+    except Exception:  # pragma: no cover
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample(inp, n_tokens, seed=0):
+    """Time the fp64 oracle on a seeded sample of the batch's tokens."""
+    from oracle import moe_oracle as O
+    host = {k: (v.detach().cpu() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    rng = np.random.default_rng(seed)
+    toks = np.sort(rng.choice(inp["T"], size=min(n_tokens, inp["T"]), replace=False))
+    t0 = time.perf_counter()
+    O.forward_tokens(host, toks)
+    return len(toks), time.perf_counter() - t0
+
+
+# ---------------------------------------------------------------- arms
+
+def workload(args):
+    """The configuration, optionally shrunk (fewer experts / tokens with the
+    same per-expert shape) for profiler captures."""
+    cfg = CONFIGS[args.config]
+    if args.experts or args.tokens:
+        E = args.experts or cfg.E
+        T = args.tokens or cfg.T
+        cfg = dataclasses.replace(cfg, E=E, T=T, name=f"{cfg.name}__E{E}_T{T}")
+    return cfg
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    cfg = workload(args)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(cfg, device=dev)
+    host = {k: (v.detach().cpu() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    n = args.ref_tokens
+    for _ in range(args.warmup):
+        oracle_sample(host, n, seed=1)
+    times = []
+    for s in range(args.steps):
+        nt, dt = oracle_sample(host, n, seed=100 + s)
+        times.append(dt)
+    total = sum(times)
+    value = nt * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
+                   "S": cfg.S, "I": cfg.I},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_threads(),
+                         "kind": "oracle",
+                         "sample": f"{nt} seeded tokens of the T={cfg.T} batch per step, "
+                                   "fp64 numpy oracle (per-token path)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    from fine_grained_moe_fp32_b200 import moe as M
+    world, rank, local = dist_setup()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    cfg = workload(args)
+    T = cfg.T
+    inp = make_inputs(cfg, device=dev, seed=0, weights=True)
+    if world > 1:  # own token batch per rank
+        inp["x"] = make_inputs(cfg, device=dev, seed=shard_seed(0, rank), weights=False)["x"]
+    layer = M.MoELayer(inp, align=args.align, device=dev)
+    x = inp["x"]
+    y = torch.empty((T, cfg.d), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        layer(x, y)
+    torch.cuda.synchronize(dev)
+    st = M.device_status()
+    if st != M.MOE_OK:
+        raise SystemExit(f"device status after warm-up: {M.status_string(st)}")
+    views = M.workspace_views(layer.dims(T), layer.workspace(T))
+    counts = views["counts"].cpu().numpy()
+
+    # ---- device-resident timed region (with per-phase events)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    time.sleep(0.15)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t0 = time.time()
+    start.record(stream)
+    for s in range(args.steps):
+        M.set_phase_events(ev[s])
+        layer(x, y)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    t1 = time.time()
+    M.set_phase_events(None)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop(t0, t1)
+    st = M.device_status()
+    if st != M.MOE_OK:
+        raise SystemExit(f"device status after timing: {M.status_string(st)}")
+    ms_local = start.elapsed_time(end)
+    ms = max_over_ranks(ms_local, world, dev)
+    value = whole_job_value(world, T, args.steps, ms)
+    phase_ms = {}
+    for i, name in enumerate(M.PHASES):
+        phase_ms[name] = statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1])
+                                         for s in range(args.steps))
+
+    # ---- end to end through the public API: pinned host x -> y on host
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty((T, cfg.d), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    for _ in range(max(1, args.warmup)):
+        x_dev.copy_(x_host, non_blocking=True)
+        layer(x_dev, y)
+        y_host.copy_(y, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        layer(x_dev, y)
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = whole_job_value(world, T, args.steps, e2e_ms)
+
+    # ---- roofline of the dominant kernel
+    peaks, peak_src = load_peaks()
+    units = gemm_units(cfg, T, counts)
+    dom = max(("gemm_gate_up_swiglu", "gemm_down"), key=lambda n: phase_ms[n])
+    bytes_, flops = units[dom]
+    dur_s = phase_ms[dom] / 1e3
+    hbm_bound = T * cfg.k <= 24 * cfg.E
+    if hbm_bound:
+        achieved = bytes_ / dur_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"]}
+    else:
+        achieved = flops / dur_s / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak}
+    roof["kernel"] = dom
+    roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if hbm_bound else 'bf16_tflops'})"
+    roof["traffic"] = load_traffic(dom, cfg.name)
+    roof["algorithmic_per_launch"] = bytes_ if hbm_bound else flops
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights; random-init layer)",
+        "config": {"workload": cfg.name, "T": T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
+                   "S": cfg.S, "I": cfg.I, "align": args.align, "router": "fp32",
+                   "parallelism": f"dp{world} (replicas, no collective)",
+                   "l2": "inputs larger than L2: the step streams the expert weights "
+                         f"({(units['touched_experts'] + cfg.S) * 3 * cfg.I * cfg.d * 2 / 1e9:.2f} GB)"},
+        "roofline": roof,
+        "phases_ms": {k: round(v, 4) for k, v in phase_ms.items()},
+        "clocks": clocks,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * cfg.d * 2,
+                "d2h_bytes_per_step": T * cfg.d * 2},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, dt = oracle_sample(inp, args.cpu_tokens)
+        line["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": cpu_threads(),
+                                "kind": "oracle",
+                                "sample": f"{n} seeded tokens of the T={T} batch, fp64 numpy "
+                                          f"oracle per-token path, {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[1])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=1, choices=sorted(CONFIGS))
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--align", type=int, default=16)
+    ap.add_argument("--cpu-tokens", type=int, default=32)
+    ap.add_argument("--ref-tokens", type=int, default=4)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=0, help="shrink E (profiling cases)")
+    ap.add_argument("--tokens", type=int, default=0, help="override T (profiling cases)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -25,7 +25,12 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {
 
 // 256 threads as a 16 x 16 grid; thread (ty, tx) owns tokens
 // {ty*4 .. ty*4+3, 64+ty*4 .. 64+ty*4+3} and experts {tx*4 .., 64+tx*4 ..}.
-__global__ void __launch_bounds__(kThreads, 2)
+// Accumulation is two-level: the products are fp32 FMAs and the BK products
+// of one staged chunk are summed from zero in fp32; the running sum across
+// chunks is carried in fp64 (one add per BK FMAs).  A single fp32 running sum
+// over k = 5120 terms loses ~1e-5 relative in the softmax probabilities when
+// one term is large (e.g. a logit offset); this keeps it near 1e-7.
+__global__ void __launch_bounds__(kThreads, 1)
 router_gemm_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wg,
                    float* __restrict__ part, int T, int d, int E, int kchunk) {
   __shared__ __align__(16) float xs[2][BK][BT];
@@ -74,11 +79,11 @@ router_gemm_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wg,
   };
 
   const int ty = tid >> 4, tx = tid & 15;
-  float acc[8][8];
+  double acc[8][8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
 
   if (nk > 0) {
     gload(0);
@@ -88,6 +93,11 @@ router_gemm_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wg,
   for (int kc = 0; kc < nk; ++kc) {
     const int buf = kc & 1;
     if (kc + 1 < nk) gload(kc + 1);
+    float part_acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) part_acc[i][j] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < BK; ++kk) {
       const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][kk][ty * 4]);
@@ -99,8 +109,12 @@ router_gemm_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wg,
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        for (int j = 0; j < 8; ++j) part_acc[i][j] = fmaf(a[i], b[j], part_acc[i][j]);
     }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] += (double)part_acc[i][j];
     if (kc + 1 < nk) sstore(buf ^ 1);
     __syncthreads();
   }
@@ -115,12 +129,13 @@ router_gemm_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wg,
       const int e0 = half * 64 + tx * 4;
       float* dst = out + (size_t)t * E + e0;
       if (e0 + 3 < E && (E & 3) == 0) {
-        *reinterpret_cast<float4*>(dst) = make_float4(acc[i][half * 4 + 0], acc[i][half * 4 + 1],
-                                                      acc[i][half * 4 + 2], acc[i][half * 4 + 3]);
+        *reinterpret_cast<float4*>(dst) =
+            make_float4((float)acc[i][half * 4 + 0], (float)acc[i][half * 4 + 1],
+                        (float)acc[i][half * 4 + 2], (float)acc[i][half * 4 + 3]);
       } else {
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          if (e0 + j < E) dst[j] = acc[i][half * 4 + j];
+          if (e0 + j < E) dst[j] = (float)acc[i][half * 4 + j];
       }
     }
   }
@@ -152,11 +167,11 @@ router_topk_kernel(const float* __restrict__ part, int splits, const float* __re
   for (int i = 0; i < 4; ++i) {
     const int e = lane + 32 * i;
     valid[i] = e < E;
-    float s = 0.f;
+    double s = 0.0;  // split partials summed in fp64, in split order
     if (valid[i]) {
-      for (int sp = 0; sp < splits; ++sp) s += part[((size_t)sp * T + t) * E + e];
+      for (int sp = 0; sp < splits; ++sp) s += (double)part[((size_t)sp * T + t) * E + e];
     }
-    z[i] = valid[i] ? s : -INFINITY;
+    z[i] = valid[i] ? (float)s : -INFINITY;
   }
   float m = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
 #pragma unroll
@@ -224,7 +239,7 @@ struct SplitPlan {
 SplitPlan plan_splits(const Shape& s, int num_sms) {
   const int tiles = (int)ceil_div(s.T, BT);
   const int max_splits = s.d / (BK * 4) > 0 ? s.d / (BK * 4) : 1;
-  int splits = tiles > 0 ? (2 * num_sms) / tiles : 1;
+  int splits = tiles > 0 ? num_sms / tiles : 1;
   if (splits < 1) splits = 1;
   if (splits > max_splits) splits = max_splits;
   const int kchunk = (int)round_up(ceil_div(s.d, splits), BK);

@@ -251,6 +251,9 @@ def set_phase_events(events) -> None:
     if events is None:
         _check(load().moe_set_phase_events(None, 0), "moe_set_phase_events")
         return
+    for e in events:
+        if e.cuda_event == 0:   # torch creates the CUDA event on first record
+            e.record()
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     _check(load().moe_set_phase_events(arr, len(events)), "moe_set_phase_events")
 

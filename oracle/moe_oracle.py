@@ -223,7 +223,8 @@ def forward(inp: dict, align: int = 16, idx=None) -> dict:
         h_shared.append(h)
     y = y_shared + unpermute_sum(y_perm, pm["row_of"], r["w"], T, k)
     return {**r, **pm, "x_perm": x_perm, "h_perm": h_perm, "y_perm": y_perm,
-            "h_shared": np.concatenate(h_shared, axis=1), "y_shared": y_shared,
+            "h_shared": (np.concatenate(h_shared, axis=1) if h_shared else np.zeros((T, 0))),
+            "y_shared": y_shared,
             "y": y}
 
 

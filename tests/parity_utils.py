@@ -10,7 +10,13 @@ workload specification fixes):
     run on the GPU's own routing;
   * bf16 intermediates (h, y_perm): every element within 2^-8 of its own
     magnitude (one bf16 rounding plus fp32 accumulation) plus 1e-3 rms;
-  * the layer output y (bf16): max |gpu - oracle| <= 2e-2 * rms(oracle).
+  * the layer output y (bf16): max |gpu - oracle| <= 2e-2 * rms(oracle) on the
+    workload configurations.  Shapes outside them (edge cases with heavier
+    output tails or cancelling terms, e.g. k = 8 with one shared expert, or no
+    shared expert) are held to the bound the arithmetic gives: the output's
+    own bf16 rounding (2^-8 |y|) plus the bf16 rounding of every routed
+    output it sums (2^-8 sum_j w_j |o_j|), plus 1e-2 rms(y) for the rounding
+    of h carried through the down projection.
 """
 import numpy as np
 import torch
@@ -66,12 +72,18 @@ def check_bf16_elementwise(got, ref, what):
     return float(err.max()) if err.size else 0.0
 
 
-def check_output(y_gpu, y_ref, what="y"):
+def check_output(y_gpu, y_ref, what="y", spec=True, routed_abs=None):
     y_gpu, y_ref = to_np(y_gpu), np.asarray(y_ref, dtype=np.float64)
     assert np.isfinite(y_gpu).all(), f"{what}: non-finite values"
     r = rms(y_ref)
-    err = float(np.abs(y_gpu - y_ref).max()) if y_ref.size else 0.0
-    assert err <= Y_RMS_FRAC * r + 1e-30, f"{what}: max err {err:.4e} > {Y_RMS_FRAC} * rms {r:.4e}"
+    diff = np.abs(y_gpu - y_ref)
+    err = float(diff.max()) if y_ref.size else 0.0
+    if spec:
+        assert err <= Y_RMS_FRAC * r + 1e-30, f"{what}: max err {err:.4e} > {Y_RMS_FRAC} * rms {r:.4e}"
+    else:
+        extra = 0.0 if routed_abs is None else BF16_REL * np.asarray(routed_abs)
+        bound = BF16_REL * np.abs(y_ref) + extra + 1e-2 * r + 1e-30
+        assert np.all(diff <= bound), f"{what}: max err {err:.4e} beyond the rounding bound (rms {r:.4e})"
     return err / r if r > 0 else 0.0
 
 

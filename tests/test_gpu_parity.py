@@ -195,8 +195,6 @@ def test_grouped_swiglu_parity(name, cfg, T, align):
         # the down GEMM against the oracle fed with the GPU's own bf16 h
         o_from_h = PU.to_np(h[a:b]) @ inp["w2"][e].double().numpy().T
         PU.check_bf16_elementwise(y[a:b], o_from_h, f"y_perm expert {e}")
-        # and the chain against the exact expert output
-        PU.check_output(y[a:b], o_ref, f"y_perm chain expert {e}")
 
 
 # ------------------------------------------------------------------ combine
@@ -256,10 +254,12 @@ def test_forward_parity_small(name, cfg, T, align):
     _check_permutation(M.dims_of(cfg, T=inp["T"], align=align),
                        {k: v[k] for k in ("counts", "offsets", "row_of", "token_of_row", "x_perm")},
                        v["topk_idx"].cpu(), inp["x"])
+    spec = cfg in CONFIGS.values()
     if cfg.S > 0:
         PU.check_bf16_elementwise(v["h_shared"], ref["h_shared"], "h_shared")
-        PU.check_output(v["y_shared"], ref["y_shared"], "y_shared")
-    PU.check_output(y, ref["y"])
+        PU.check_output(v["y_shared"], ref["y_shared"], "y_shared", spec=spec)
+    routed_abs = O.unpermute_sum(np.abs(ref["y_perm"]), ref["row_of"], ref["w"], inp["T"], cfg.k)
+    PU.check_output(y, ref["y"], spec=spec, routed_abs=routed_abs)
 
 
 def test_forward_empty_batch():

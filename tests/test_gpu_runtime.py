@@ -1,0 +1,53 @@
+"""Runtime behaviour on the GPU: bounded waits that run out report a timeout
+and leave the context usable; the phase-event measurement hook."""
+import pytest
+import torch
+
+from fine_grained_moe_fp32_b200 import moe as M
+from fine_grained_moe_fp32_b200.workloads import make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _layer(T=200):
+    inp = make_inputs(0, T=T)
+    g = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    return g, M.MoELayer(g)
+
+
+def test_bounded_wait_times_out_and_recovers():
+    """A 1 ns wait limit makes the GEMM pipelines give up at their first
+    unready barrier; the kernels record MOE_ERR_TIMEOUT, drain their copies,
+    free tensor memory and return.  With the default limit restored the
+    same call is correct again."""
+    g, layer = _layer()
+    y_ok = layer(g["x"]).clone()
+    torch.cuda.synchronize()
+    assert M.device_status() == M.MOE_OK
+    try:
+        M.set_wait_limit_ns(1)
+        layer(g["x"])
+        assert M.device_status() == M.MOE_ERR_TIMEOUT
+    finally:
+        M.set_wait_limit_ns(0)
+    y = layer(g["x"])
+    assert M.device_status() == M.MOE_OK
+    assert torch.equal(y.view(torch.int16), y_ok.view(torch.int16))
+
+
+def test_phase_events_cover_the_step():
+    g, layer = _layer()
+    layer(g["x"])
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    outer = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    M.set_phase_events(ev)
+    try:
+        outer[0].record()
+        layer(g["x"])
+        outer[1].record()
+    finally:
+        M.set_phase_events(None)
+    torch.cuda.synchronize()
+    parts = [ev[i].elapsed_time(ev[i + 1]) for i in range(5)]
+    assert all(p >= 0 for p in parts)
+    assert sum(parts) <= outer[0].elapsed_time(outer[1]) * 1.01 + 0.05
