@@ -26,7 +26,7 @@ EXPORTED = (
     "moe_capacity", "moe_status_string", "moe_route_workspace_size", "moe_route",
     "moe_permute_workspace_size", "moe_permute", "moe_grouped_swiglu", "moe_combine",
     "moe_workspace_size", "moe_forward_layout", "moe_forward", "moe_get_last_device_status",
-    "moe_set_wait_limit_ns", "moe_set_phase_events",
+    "moe_set_wait_limit_ns", "moe_set_phase_events", "moe_route_noalloc",
 )
 
 
@@ -77,6 +77,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_get_last_device_status": (I, [V]),
         "moe_set_wait_limit_ns": (I, [ctypes.c_uint64]),
         "moe_set_phase_events": (I, [ctypes.POINTER(ctypes.c_void_p), I]),
+        "moe_route_noalloc": (I, [P, V, V, V, V, V, V, V]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -168,6 +169,20 @@ def route(dm, x, w_gate, bias, probs, topk_idx, topk_w, workspace, stream=None):
                           _ptr(topk_idx), _ptr(topk_w), _ptr(workspace),
                           workspace.numel() if workspace is not None else 0, _stream(stream))
     _check(rc, "moe_route")
+
+
+def route_noalloc(dm, x, w_gate, bias, probs, topk_idx, topk_w, stream=None):
+    """moe_route for callers that cannot allocate device memory: the scratch
+    is a fixed 16 MiB array inside the library (see include/moe_b200.h)."""
+    _expect(x, torch.bfloat16, (dm.T, dm.d), "x")
+    _expect(w_gate, torch.float32, (dm.E, dm.d), "w_gate")
+    _expect(bias, torch.float32, (dm.E,), "bias")
+    _expect(probs, torch.float32, (dm.T, dm.E), "probs")
+    _expect(topk_idx, torch.int32, (dm.T, dm.k), "topk_idx")
+    _expect(topk_w, torch.float32, (dm.T, dm.k), "topk_w")
+    rc = load().moe_route_noalloc(ctypes.byref(dm), _ptr(x), _ptr(w_gate), _ptr(bias),
+                                  _ptr(probs), _ptr(topk_idx), _ptr(topk_w), _stream(stream))
+    _check(rc, "moe_route_noalloc")
 
 
 def permute(dm, topk_idx, x, counts, offsets, row_of, token_of_row, x_perm, workspace,

@@ -96,6 +96,31 @@ int moe_route(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
               void* stream);
 
 /* ------------------------------------------------------------------------
+ * moe_route_noalloc -- moe_route without a caller workspace.
+ * The pages have no counterpart of this call; it exists for callers that
+ * cannot allocate device memory when they route -- an inference engine's
+ * plugin/enqueue hook that is handed a stream and its buffers but no
+ * allocator, or a serving loop that forbids allocation after warm-up because
+ * cudaMalloc can synchronise the device and fragments a pool owned by someone
+ * else.  It allocates nothing: the split-K partial logits live in a fixed
+ * 16 MiB array inside the library, which every GPU that loads the library
+ * holds until the process exits.
+ *
+ * Arguments and results are those of moe_route (same kernels, bit-identical
+ * output).  Shapes whose partials need more than 16 MiB
+ * (moe_route_workspace_size(dims) > 16 MiB, e.g. E = 128 beyond ~30k
+ * tokens) are rejected with MOE_ERR_WORKSPACE before anything is launched.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the array: it needs no clearing (every partial
+ * read is written first in the same call), but calls that overlap on the GPU
+ * (other streams, other host threads on the same device) race on it.
+ * ---------------------------------------------------------------------- */
+int moe_route_noalloc(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
+                      const float* bias, float* probs, int32_t* topk_idx,
+                      float* topk_w, void* stream);
+
+/* ------------------------------------------------------------------------
  * moe_permute -- counting sort of the (token, slot) pairs into per-expert
  * segments padded to `align` rows, and the row gather of x.
  * Technical Report, Method (systems paragraph): expert segments are padded to
