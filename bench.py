@@ -38,6 +38,7 @@ from fine_grained_moe_fp32_b200.workloads import CONFIGS, make_inputs  # noqa: E
 METRIC = "MoE-layer tokens/s (bf16, d=5120, 128E top-6 + 2 shared) and % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNELS_PER_STEP = 9  # router gemm + top-k, 4 permutation kernels, 2 grouped GEMMs, combine
+BWD_KERNELS = 12      # combine/router bwd (3), 5 grouped GEMMs, 2 gate GEMMs + split sum, un-permute
 
 
 # ---------------------------------------------------------------- helpers
@@ -169,6 +170,16 @@ def shard_seed(seed: int, rank: int) -> int:
     return seed + 7919 * rank
 
 
+def train_gemm_flops(cfg, T):
+    """Algorithmic flops of each grouped-GEMM phase of one fwd+bwd step."""
+    d, I, S, k = cfg.d, cfg.I, cfg.S, cfg.k
+    rows = T * k
+    up = 2 * (rows * 2 * I + T * 2 * S * I) * d      # gate/up shaped
+    down = 2 * (rows * I + T * S * I) * d            # down shaped
+    return {"gemm_gate_up_swiglu": up, "gemm_down": down, "dgrad_down_swiglu_bwd": down,
+            "wgrad_w2": down, "dgrad_up": up, "wgrad_w1_w3": up}
+
+
 def gemm_units(cfg, T, counts):
     """Algorithmic work of the two grouped GEMMs for one step (padding not
     counted): bytes that must move and flops that must be done."""
@@ -195,13 +206,23 @@ def cpu_threads():
 
 
 def oracle_sample(inp, n_tokens, seed=0):
-    """Time the fp64 oracle on a seeded sample of the batch's tokens."""
+    """Time the fp64 oracle on a seeded sample of the batch's tokens: the
+    forward (per-token path), or for a training workload the forward and the
+    backward of the sampled tokens (input gradients, router and all experts;
+    weight gradients not kept)."""
     from oracle import moe_oracle as O
     host = {k: (v.detach().cpu() if torch.is_tensor(v) else v) for k, v in inp.items()}
     rng = np.random.default_rng(seed)
     toks = np.sort(rng.choice(inp["T"], size=min(n_tokens, inp["T"]), replace=False))
     t0 = time.perf_counter()
-    O.forward_tokens(host, toks)
+    if inp["cfg"].grad:
+        sub = dict(host)
+        idx = torch.as_tensor(toks)
+        sub["x"], sub["dy"], sub["T"] = host["x"][idx], host["dy"][idx], len(toks)
+        f = O.forward(sub)
+        O.backward(sub, sub["dy"], f, experts=[])
+    else:
+        O.forward_tokens(host, toks)
     return len(toks), time.perf_counter() - t0
 
 
@@ -274,18 +295,33 @@ def run_ours(args):
     x = inp["x"]
     y = torch.empty((T, cfg.d), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
+    train = cfg.grad
+    if train:
+        dy = inp["dy"]
+        grads = layer.alloc_grads(T)
+
+        def step(xin, yout):
+            layer.forward_train(xin, yout)
+            layer.backward(xin, dy, grads)
+    else:
+        def step(xin, yout):
+            layer(xin, yout)
+    n_events = 13 if train else 6
+    phase_names = M.PHASES + (M.BWD_PHASES if train else ())
 
     for _ in range(args.warmup):
-        layer(x, y)
+        step(x, y)
     torch.cuda.synchronize(dev)
     st = M.device_status()
     if st != M.MOE_OK:
         raise SystemExit(f"device status after warm-up: {M.status_string(st)}")
-    views = M.workspace_views(layer.dims(T), layer.workspace(T))
+    views = M.workspace_views(layer.dims(T), layer.train_workspace(T) if train
+                              else layer.workspace(T))
     counts = views["counts"].cpu().numpy()
 
     # ---- device-resident timed region (with per-phase events)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_events)]
+          for _ in range(args.steps)]
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
@@ -297,7 +333,7 @@ def run_ours(args):
     start.record(stream)
     for s in range(args.steps):
         M.set_phase_events(ev[s])
-        layer(x, y)
+        step(x, y)
     end.record(stream)
     torch.cuda.synchronize(dev)
     t1 = time.time()
@@ -315,15 +351,30 @@ def run_ours(args):
     for i, name in enumerate(M.PHASES):
         phase_ms[name] = statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1])
                                          for s in range(args.steps))
+    for i, name in enumerate(M.BWD_PHASES if train else ()):
+        phase_ms[name] = statistics.mean(ev[s][6 + i].elapsed_time(ev[s][7 + i])
+                                         for s in range(args.steps))
 
     # ---- end to end through the public API: pinned host x -> y on host
     x_host = x.cpu().pin_memory()
     y_host = torch.empty((T, cfg.d), dtype=torch.bfloat16).pin_memory()
     x_dev = torch.empty_like(x)
+    if train:
+        dy_host = dy.cpu().pin_memory()
+        dy_dev = dy
+
+        def e2e_step():
+            x_dev.copy_(x_host, non_blocking=True)
+            dy_dev.copy_(dy_host, non_blocking=True)
+            step(x_dev, y)
+            y_host.copy_(grads["dx"], non_blocking=True)
+    else:
+        def e2e_step():
+            x_dev.copy_(x_host, non_blocking=True)
+            step(x_dev, y)
+            y_host.copy_(y, non_blocking=True)
     for _ in range(max(1, args.warmup)):
-        x_dev.copy_(x_host, non_blocking=True)
-        layer(x_dev, y)
-        y_host.copy_(y, non_blocking=True)
+        e2e_step()
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
@@ -331,9 +382,7 @@ def run_ours(args):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        layer(x_dev, y)
-        y_host.copy_(y, non_blocking=True)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
@@ -342,10 +391,15 @@ def run_ours(args):
     # ---- roofline of the dominant kernel
     peaks, peak_src = load_peaks()
     units = gemm_units(cfg, T, counts)
-    dom = max(("gemm_gate_up_swiglu", "gemm_down"), key=lambda n: phase_ms[n])
-    bytes_, flops = units[dom]
+    if train:
+        tflops = train_gemm_flops(cfg, T)
+        dom = max(tflops, key=lambda n: phase_ms[n])
+        bytes_, flops = 0, tflops[dom]
+    else:
+        dom = max(("gemm_gate_up_swiglu", "gemm_down"), key=lambda n: phase_ms[n])
+        bytes_, flops = units[dom]
     dur_s = phase_ms[dom] / 1e3
-    hbm_bound = T * cfg.k <= 24 * cfg.E
+    hbm_bound = (not train) and T * cfg.k <= 24 * cfg.E
     if hbm_bound:
         achieved = bytes_ / dur_s / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
@@ -373,16 +427,21 @@ def run_ours(args):
         "roofline": roof,
         "phases_ms": {k: round(v, 4) for k, v in phase_ms.items()},
         "clocks": clocks,
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * cfg.d * 2,
+        "e2e": {"value": e2e_value, "unit": "tokens/s",
+                "h2d_bytes_per_step": T * cfg.d * 2 * (2 if train else 1),
                 "d2h_bytes_per_step": T * cfg.d * 2},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": (KERNELS_PER_STEP + (BWD_KERNELS if train else 0)) * args.steps,
     }
+    if train:
+        line["config"]["step"] = "forward (training, keeps g/u) + backward"
+        line["train_tflop_per_step"] = sum(train_gemm_flops(cfg, T).values()) / 1e12
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n, dt = oracle_sample(inp, args.cpu_tokens)
         line["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": cpu_threads(),
                                 "kind": "oracle",
                                 "sample": f"{n} seeded tokens of the T={T} batch, fp64 numpy "
-                                          f"oracle per-token path, {dt:.1f} s"}
+                                          f"oracle ({'forward + backward' if train else 'forward'}"
+                                          f"), {dt:.1f} s"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -1,0 +1,328 @@
+// Backward of the MoE layer outside the expert GEMMs (selection held fixed;
+// the bias only enters the selection key and gets no gradient):
+//
+//   combine_bwd_kernel     dy_perm[row(t,j)] = w[t,j] * dy[t];  dw[t,j] = <dy[t], y_perm[row(t,j)]>
+//   zero_padding_rows      dy_perm padding rows = 0 (the wgrad sums run over them)
+//   router_bwd_kernel      renormalisation and softmax backward, one warp per token:
+//                          dp_j = (dw_j - sum_i w_i dw_i) / sum_sel p;
+//                          dz_e = p_e (dp_e - sum_e' p_e' dp_e')  (dp = 0 off the chosen experts)
+//   sgemm_kernel           fp32 GEMMs on CUDA cores for the gate: dz Wg (-> dx) and
+//                          dz^T x (-> dWg, split-K partials summed in order)
+//   unpermute_bwd_kernel   dx[t] = dx_shared[t] + dz Wg [t] + sum_j dx_perm[row(t,j)]
+#include <cuda_bf16.h>
+
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+}
+
+constexpr int kCbThreads = 128;
+constexpr int kMaxVecPerThread = 8;  // d <= 8 * 8 * 128 = 8192
+
+// One CTA per token.  The dot products are reduced in a fixed order (per
+// thread, then warp butterfly, then warps in order), so dw is deterministic.
+__global__ void __launch_bounds__(kCbThreads)
+combine_bwd_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ y_perm,
+                   const int32_t* __restrict__ row_of, const float* __restrict__ topk_w,
+                   uint16_t* __restrict__ dy_perm, float* __restrict__ dw, int d, int k,
+                   int64_t cap) {
+  const int t = blockIdx.x;
+  __shared__ float red[kCbThreads / 32];
+  const int nv = d / 8;
+  uint4 g[kMaxVecPerThread];
+#pragma unroll
+  for (int i = 0; i < kMaxVecPerThread; ++i) {
+    const int v = threadIdx.x + i * kCbThreads;
+    g[i] = v < nv ? reinterpret_cast<const uint4*>(dy + (size_t)t * d)[v] : make_uint4(0, 0, 0, 0);
+  }
+  for (int j = 0; j < k; ++j) {
+    const int r = row_of[(size_t)t * k + j];
+    const float w = topk_w[(size_t)t * k + j];
+    float part = 0.f;
+    if (r >= 0 && r < cap) {
+      const uint4* yr = reinterpret_cast<const uint4*>(y_perm + (size_t)r * d);
+      uint4* out = reinterpret_cast<uint4*>(dy_perm + (size_t)r * d);
+#pragma unroll
+      for (int i = 0; i < kMaxVecPerThread; ++i) {
+        const int v = threadIdx.x + i * kCbThreads;
+        if (v < nv) {
+          const uint4 yv = yr[v];
+          const uint32_t gw[4] = {g[i].x, g[i].y, g[i].z, g[i].w};
+          const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            part = fmaf(bf16lo(gw[q]), bf16lo(yw[q]), part);
+            part = fmaf(bf16hi(gw[q]), bf16hi(yw[q]), part);
+            o[q] = pack_bf16(w * bf16lo(gw[q]), w * bf16hi(gw[q]));
+          }
+          out[v] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = part;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float s = 0.f;
+      for (int i = 0; i < kCbThreads / 32; ++i) s += red[i];
+      dw[(size_t)t * k + j] = s;
+    }
+    __syncthreads();
+  }
+}
+
+constexpr int kPadWarps = 8;
+
+__global__ void __launch_bounds__(kPadWarps * 32)
+zero_padding_rows_kernel(uint16_t* __restrict__ rows, int d, const int32_t* __restrict__ offsets,
+                         int E, const int32_t* __restrict__ token_of_row, int64_t cap) {
+  const int64_t r = (int64_t)blockIdx.x * kPadWarps + (threadIdx.x >> 5);
+  if (r >= cap || r >= offsets[E] || token_of_row[r] >= 0) return;
+  uint4* dst = reinterpret_cast<uint4*>(rows + (size_t)r * d);
+  for (int v = threadIdx.x & 31; v < d / 8; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+}
+
+constexpr int kRbWarps = 8;
+
+__global__ void __launch_bounds__(kRbWarps * 32)
+router_bwd_kernel(const float* __restrict__ probs, const int32_t* __restrict__ topk_idx,
+                  const float* __restrict__ topk_w, const float* __restrict__ dw,
+                  float* __restrict__ dz, int T, int E, int k) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kRbWarps + (threadIdx.x >> 5);
+  if (t >= T) return;
+  // chosen experts, their probabilities and weight gradients (lane j < k)
+  int e_j = 0;
+  float p_j = 0.f, w_j = 0.f, dw_j = 0.f;
+  if (lane < k) {
+    e_j = topk_idx[(size_t)t * k + lane];
+    e_j = min(max(e_j, 0), E - 1);
+    p_j = probs[(size_t)t * E + e_j];
+    w_j = topk_w[(size_t)t * k + lane];
+    dw_j = dw[(size_t)t * k + lane];
+  }
+  float psum = 0.f, wdw = 0.f;
+  for (int j = 0; j < k; ++j) {  // fixed order
+    psum += __shfl_sync(0xffffffffu, p_j, j);
+    wdw += __shfl_sync(0xffffffffu, w_j * dw_j, j);
+  }
+  const float dp_j = lane < k ? (dw_j - wdw) / psum : 0.f;
+  float pdp = 0.f;
+  for (int j = 0; j < k; ++j) pdp += __shfl_sync(0xffffffffu, p_j * dp_j, j);
+  for (int i = 0; i < 4; ++i) {
+    const int e = lane + 32 * i;
+    if (e >= E) break;
+    float dpe = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int ej = __shfl_sync(0xffffffffu, e_j, j);
+      const float dpj = __shfl_sync(0xffffffffu, dp_j, j);
+      if (ej == e) dpe = dpj;
+    }
+    const float pe = probs[(size_t)t * E + e];
+    dz[(size_t)t * E + e] = pe * (dpe - pdp);
+  }
+}
+
+// fp32 GEMM on CUDA cores: C[m, n] (+)= sum_k A(m, k) B(k, n).
+//   A(m, k) = a[m * lda + k]  (A_MMAJOR = false)  or  a[k * lda + m]  (true)
+//   B(k, n) = b[k * ldb + n]  (TB = float or bf16 bits)
+// 128 x 128 tile, 16-deep k chunks in smem, 16 x 16 threads of 8 x 8
+// outputs; fp32 chunk sums added into an fp64 running sum.  blockIdx.z is the
+// split of K; each split writes its own partial C slab.
+constexpr int SB = 128, SK = 16, kSgThreads = 256;
+
+template <bool A_MMAJOR, typename TB>
+__global__ void __launch_bounds__(kSgThreads, 1)
+sgemm_kernel(const float* __restrict__ a, int lda, const TB* __restrict__ b, int ldb,
+             float* __restrict__ c, int ldc, int64_t c_split_stride, int M, int N, int K,
+             int kchunk) {
+  __shared__ __align__(16) float As[SK][SB];
+  __shared__ __align__(16) float Bs[SK][SB];
+  const int tid = threadIdx.x;
+  const int m0 = blockIdx.y * SB, n0 = blockIdx.x * SB;
+  const int k_begin = blockIdx.z * kchunk;
+  const int k_end = min(K, k_begin + kchunk);
+  const int ty = tid >> 4, tx = tid & 15;
+  double acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+
+  for (int k0 = k_begin; k0 < k_end; k0 += SK) {
+    // ---- stage A (128 m x 16 k) into As[k][m]
+    if (A_MMAJOR) {
+      for (int i = tid; i < SK * SB; i += kSgThreads) {
+        const int kk = i / SB, mm = i % SB;
+        const int gm = m0 + mm, gk = k0 + kk;
+        As[kk][mm] = (gm < M && gk < k_end) ? a[(size_t)gk * lda + gm] : 0.f;
+      }
+    } else {
+      for (int i = tid; i < SK * SB; i += kSgThreads) {
+        const int mm = i / SK, kk = i % SK;
+        const int gm = m0 + mm, gk = k0 + kk;
+        As[kk][mm] = (gm < M && gk < k_end) ? a[(size_t)gm * lda + gk] : 0.f;
+      }
+    }
+    // ---- stage B (16 k x 128 n) into Bs[k][n]
+    for (int i = tid; i < SK * SB; i += kSgThreads) {
+      const int kk = i / SB, nn = i % SB;
+      const int gk = k0 + kk, gn = n0 + nn;
+      float v = 0.f;
+      if (gk < k_end && gn < N) {
+        if constexpr (sizeof(TB) == 2)
+          v = __uint_as_float((uint32_t)b[(size_t)gk * ldb + gn] << 16);
+        else
+          v = b[(size_t)gk * ldb + gn];
+      }
+      Bs[kk][nn] = v;
+    }
+    __syncthreads();
+    float part[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) part[i][j] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < SK; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][64 + tx * 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) part[i][j] = fmaf(av[i], bv[j], part[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] += (double)part[i][j];
+    __syncthreads();
+  }
+  float* cs = c + (size_t)blockIdx.z * c_split_stride;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int gm = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
+    if (gm >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int gn = n0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + (j - 4));
+      if (gn < N) cs[(size_t)gm * ldc + gn] = (float)acc[i][j];
+    }
+  }
+}
+
+__global__ void sum_splits_kernel(const float* __restrict__ part, int splits, int64_t n,
+                                  float* __restrict__ out) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  double s = 0.0;
+  for (int sp = 0; sp < splits; ++sp) s += (double)part[(size_t)sp * n + i];
+  out[i] = (float)s;
+}
+
+__global__ void __launch_bounds__(kCbThreads)
+unpermute_bwd_kernel(const float* __restrict__ dx_shared, const float* __restrict__ dx_router,
+                     const float* __restrict__ dx_perm, const int32_t* __restrict__ row_of,
+                     uint16_t* __restrict__ dx, int d, int k, int64_t cap) {
+  const int t = blockIdx.x;
+  __shared__ int rows[8];
+  if (threadIdx.x < k) {
+    const int r = row_of[(size_t)t * k + threadIdx.x];
+    rows[threadIdx.x] = (r >= 0 && r < cap) ? r : -1;
+  }
+  __syncthreads();
+  for (int v = threadIdx.x; v < d / 8; v += kCbThreads) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    if (dx_shared != nullptr) {
+      const float4* s = reinterpret_cast<const float4*>(dx_shared + (size_t)t * d) + 2 * v;
+      const float4 p0 = s[0], p1 = s[1];
+      acc[0] = p0.x; acc[1] = p0.y; acc[2] = p0.z; acc[3] = p0.w;
+      acc[4] = p1.x; acc[5] = p1.y; acc[6] = p1.z; acc[7] = p1.w;
+    }
+    {
+      const float4* s = reinterpret_cast<const float4*>(dx_router + (size_t)t * d) + 2 * v;
+      const float4 p0 = s[0], p1 = s[1];
+      acc[0] += p0.x; acc[1] += p0.y; acc[2] += p0.z; acc[3] += p0.w;
+      acc[4] += p1.x; acc[5] += p1.y; acc[6] += p1.z; acc[7] += p1.w;
+    }
+    for (int j = 0; j < k; ++j) {
+      if (rows[j] < 0) continue;
+      const float4* src = reinterpret_cast<const float4*>(dx_perm + (size_t)rows[j] * d) + 2 * v;
+      const float4 p0 = src[0], p1 = src[1];
+      acc[0] += p0.x; acc[1] += p0.y; acc[2] += p0.z; acc[3] += p0.w;
+      acc[4] += p1.x; acc[5] += p1.y; acc[6] += p1.z; acc[7] += p1.w;
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) o[q] = pack_bf16(acc[2 * q], acc[2 * q + 1]);
+    reinterpret_cast<uint4*>(dx + (size_t)t * d)[v] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+}  // namespace
+
+int dwg_splits(const Shape& s) {
+  const int tiles = (int)ceil_div(s.d, SB) * (int)ceil_div(s.E, SB);
+  int sp = tiles > 0 ? 148 / tiles : 1;
+  sp = sp < 1 ? 1 : sp;
+  const int max_sp = s.T / 256 > 0 ? s.T / 256 : 1;
+  return sp > max_sp ? max_sp : sp;
+}
+
+cudaError_t launch_backward_misc_pre(const Shape& s, const BackwardMiscArgs& a, cudaStream_t st) {
+  if (s.T > 0) {
+    combine_bwd_kernel<<<s.T, kCbThreads, 0, st>>>(a.dy, a.y_perm, a.row_of, a.topk_w, a.dy_perm,
+                                                   a.dw, s.d, s.k, s.cap);
+    router_bwd_kernel<<<(unsigned)ceil_div(s.T, kRbWarps), kRbWarps * 32, 0, st>>>(
+        a.probs, a.topk_idx, a.topk_w, a.dw, a.dz, s.T, s.E, s.k);
+  }
+  if (s.cap > 0)
+    zero_padding_rows_kernel<<<(unsigned)ceil_div(s.cap, kPadWarps), kPadWarps * 32, 0, st>>>(
+        a.dy_perm, s.d, a.offsets, s.E, a.token_of_row, s.cap);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_backward_misc_post(const Shape& s, const BackwardMiscArgs& a,
+                                      cudaStream_t st) {
+  if (s.T == 0) {
+    return cudaMemsetAsync(a.dw_gate, 0, (size_t)s.E * s.d * sizeof(float), st);
+  }
+  // dz Wg -> dx_router [T, d]   (A = dz [T, E] K-major, B = Wg [E, d])
+  {
+    dim3 grid((unsigned)ceil_div(s.d, SB), (unsigned)ceil_div(s.T, SB), 1);
+    sgemm_kernel<false, float><<<grid, kSgThreads, 0, st>>>(a.dz, s.E, a.w_gate, s.d, a.dx_router,
+                                                            s.d, 0, s.T, s.d, s.E, s.E);
+  }
+  // dz^T x -> dWg [E, d]   (A(e, t) = dz[t, e], B = x [T, d] bf16), split-K over tokens
+  {
+    const int sp = dwg_splits(s);
+    const int kchunk = (int)round_up(ceil_div(s.T, sp), SK);
+    const int splits = (int)ceil_div(s.T, kchunk);
+    dim3 grid((unsigned)ceil_div(s.d, SB), (unsigned)ceil_div(s.E, SB), (unsigned)splits);
+    sgemm_kernel<true, uint16_t><<<grid, kSgThreads, 0, st>>>(
+        a.dz, s.E, a.x, s.d, a.dwg_partials, s.d, (int64_t)s.E * s.d, s.E, s.d, s.T, kchunk);
+    const int64_t n = (int64_t)s.E * s.d;
+    sum_splits_kernel<<<(unsigned)ceil_div(n, 256), 256, 0, st>>>(a.dwg_partials, splits, n,
+                                                                   a.dw_gate);
+  }
+  unpermute_bwd_kernel<<<s.T, kCbThreads, 0, st>>>(a.dx_shared, a.dx_router, a.dx_perm, a.row_of,
+                                                   a.dx, s.d, s.k, s.cap);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -61,6 +61,12 @@ struct GemmParams {
   void* out_shared;
   int ld_shared;
   int shared_f32;
+  // gate/up GEMM only, training: also store the pre-activations g = W1 x and
+  // u = W3 x (bf16, same layout as h) for the backward pass; null = skip
+  uint16_t* g_routed;
+  uint16_t* u_routed;
+  uint16_t* g_shared;
+  uint16_t* u_shared;
   unsigned int* status;
   uint64_t wait_limit_ns;
 };
@@ -376,6 +382,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r,
                     __bfloat16_as_ushort(__float2bfloat16_rn(h));
               }
             }
+            uint16_t* gs = routed ? p.g_routed : p.g_shared;
+            uint16_t* us = routed ? p.u_routed : p.u_shared;
+            if (gs != nullptr) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                if (j < nj) {
+                  const size_t at = (size_t)(ti.row0 + c0 + j) * ld + col;
+                  gs[at] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+                  us[at] = __bfloat16_as_ushort(__float2bfloat16_rn(up_buf[j * 64 + frow]));
+                }
+              }
+            }
           }
           named_bar_sync(1, kEpiThreads);
         }
@@ -485,6 +503,10 @@ cudaError_t launch_grouped_gemms(const Shape& s, const GroupedGemmArgs& a, int n
     p.out_shared = a.h_shared;
     p.ld_shared = s.S * s.I;
     p.shared_f32 = 0;
+    p.g_routed = a.g_perm;
+    p.u_routed = a.u_perm;
+    p.g_shared = shared ? a.g_shared : nullptr;
+    p.u_shared = shared ? a.u_shared : nullptr;
     p.status = status;
     p.wait_limit_ns = wait_limit_ns;
     cudaError_t err = small ? launch_one<kSwiGLU, 32, 10>(m, p, num_sms, st)

@@ -17,11 +17,17 @@ constexpr int kMaxDevices = 64;
 constexpr int kPlanSMs = 148;  // split-K planning of the router is device independent
 constexpr uint64_t kDefaultWaitNs = 1000000000ull;
 uint64_t g_wait_limit_ns = kDefaultWaitNs;
-cudaEvent_t g_phase_events[6] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
-bool g_phase_on = false;
+constexpr int kFwdEvents = 6, kAllEvents = 13;
+cudaEvent_t g_phase_events[kAllEvents] = {};
+bool g_phase_on = false;       // forward events set
+bool g_bwd_phase_on = false;   // backward events set too
 
 cudaError_t phase(int i, cudaStream_t st) {
   return g_phase_on ? cudaEventRecord(g_phase_events[i], st) : cudaSuccess;
+}
+
+cudaError_t bwd_phase(int i, cudaStream_t st) {
+  return g_bwd_phase_on ? cudaEventRecord(g_phase_events[kFwdEvents + i], st) : cudaSuccess;
 }
 
 struct DeviceInfo {
@@ -89,6 +95,33 @@ moe_ws_layout make_layout(const Shape& s) {
   L.y_perm = take((size_t)s.cap * s.d * 2);
   L.h_shared = take((size_t)s.T * s.S * s.I * 2);
   L.y_shared = take((size_t)s.T * s.d * 4);
+  L.total = off;
+  return L;
+}
+
+moe_train_layout make_train_layout(const Shape& s) {
+  moe_train_layout L{};
+  L.fwd = make_layout(s);
+  size_t off = L.fwd.total;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += al256(bytes);
+    return at;
+  };
+  const size_t SI = (size_t)s.S * s.I;
+  L.g_perm = take((size_t)s.cap * s.I * 2);
+  L.u_perm = take((size_t)s.cap * s.I * 2);
+  L.g_shared = take((size_t)s.T * SI * 2);
+  L.u_shared = take((size_t)s.T * SI * 2);
+  L.dy_perm = take((size_t)s.cap * s.d * 2);
+  L.dw = take((size_t)s.T * s.k * 4);
+  L.dz = take((size_t)s.T * s.E * 4);
+  L.dgu_perm = take((size_t)s.cap * 2 * s.I * 2);
+  L.dgu_shared = take((size_t)s.T * 2 * SI * 2);
+  L.dx_perm = take((size_t)s.cap * s.d * 4);
+  L.dx_shared = take((size_t)s.T * s.d * 4);
+  L.dx_router = take((size_t)s.T * s.d * 4);
+  L.dwg_partials = take((size_t)dwg_splits(s) * s.E * s.d * 4);
   L.total = off;
   return L;
 }
@@ -229,10 +262,16 @@ int moe_forward_layout(const moe_dims* dims, moe_ws_layout* layout) {
   return MOE_OK;
 }
 
-int moe_forward(const moe_dims* dims, const moe_bf16* x, const float* w_gate, const float* bias,
-                const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2, const moe_bf16* ws1,
-                const moe_bf16* ws3, const moe_bf16* ws2, moe_bf16* y, void* workspace,
-                size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace moe {
+namespace {
+
+// The fused forward; with `train` it also stores the gate/up pre-activations.
+int forward_impl(const moe_dims* dims, const moe_bf16* x, const float* w_gate, const float* bias,
+                 const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2, const moe_bf16* ws1,
+                 const moe_bf16* ws3, const moe_bf16* ws2, moe_bf16* y, void* workspace,
+                 size_t workspace_bytes, void* stream, bool train) {
   Shape s;
   int rc = check_dims(dims, &s);
   if (rc != MOE_OK) return rc;
@@ -244,8 +283,10 @@ int moe_forward(const moe_dims* dims, const moe_bf16* x, const float* w_gate, co
       !aligned(w2, 16) || !aligned(y, 16) || !aligned(ws1, 16) || !aligned(ws3, 16) ||
       !aligned(ws2, 16))
     return MOE_ERR_INVALID_ARG;
-  const moe_ws_layout L = make_layout(s);
-  if (workspace == nullptr || workspace_bytes < L.total || !aligned(workspace, 256))
+  const moe_train_layout TL = make_train_layout(s);
+  const moe_ws_layout& L = TL.fwd;
+  const size_t need = train ? TL.total : L.total;
+  if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256))
     return MOE_ERR_WORKSPACE;
   const DeviceInfo* di = device_info();
   if (di == nullptr) return MOE_ERR_CUDA;
@@ -291,12 +332,149 @@ int moe_forward(const moe_dims* dims, const moe_bf16* x, const float* w_gate, co
     a.h_shared = h_sh;
     a.y_shared = y_sh;
   }
+  if (train) {
+    a.g_perm = at<uint16_t>(ws, TL.g_perm);
+    a.u_perm = at<uint16_t>(ws, TL.u_perm);
+    a.g_shared = at<uint16_t>(ws, TL.g_shared);
+    a.u_shared = at<uint16_t>(ws, TL.u_shared);
+  }
   e = launch_grouped_gemms(s, a, di->num_sms, di->status, g_wait_limit_ns, st,
                            g_phase_on ? g_phase_events[3] : nullptr);
   if (e == cudaSuccess) e = phase(4, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   e = launch_combine(s, y_perm, row_of, wts, s.S > 0 ? y_sh : nullptr, y, st);
   if (e == cudaSuccess) e = phase(5, st);
+  return cuda_status(e);
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+int moe_forward(const moe_dims* dims, const moe_bf16* x, const float* w_gate, const float* bias,
+                const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2, const moe_bf16* ws1,
+                const moe_bf16* ws3, const moe_bf16* ws2, moe_bf16* y, void* workspace,
+                size_t workspace_bytes, void* stream) {
+  return forward_impl(dims, x, w_gate, bias, w1, w3, w2, ws1, ws3, ws2, y, workspace,
+                      workspace_bytes, stream, false);
+}
+
+size_t moe_train_workspace_size(const moe_dims* dims) {
+  Shape s;
+  if (check_dims(dims, &s) != MOE_OK) return 0;
+  return make_train_layout(s).total;
+}
+
+int moe_train_layout_of(const moe_dims* dims, moe_train_layout* layout) {
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != MOE_OK) return rc;
+  if (layout == nullptr) return MOE_ERR_INVALID_ARG;
+  *layout = make_train_layout(s);
+  return MOE_OK;
+}
+
+int moe_forward_train(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
+                      const float* bias, const moe_bf16* w1, const moe_bf16* w3,
+                      const moe_bf16* w2, const moe_bf16* ws1, const moe_bf16* ws3,
+                      const moe_bf16* ws2, moe_bf16* y, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != MOE_OK) return rc;
+  if (s.I % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return forward_impl(dims, x, w_gate, bias, w1, w3, w2, ws1, ws3, ws2, y, workspace,
+                      workspace_bytes, stream, true);
+}
+
+int moe_backward(const moe_dims* dims, const moe_bf16* x, const float* w_gate, const moe_bf16* w1,
+                 const moe_bf16* w3, const moe_bf16* w2, const moe_bf16* ws1, const moe_bf16* ws3,
+                 const moe_bf16* ws2, const moe_bf16* dy, void* workspace, size_t workspace_bytes,
+                 moe_bf16* dx, float* dw_gate, moe_bf16* dw1, moe_bf16* dw3, moe_bf16* dw2,
+                 moe_bf16* dws1, moe_bf16* dws3, moe_bf16* dws2, void* stream) {
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != MOE_OK) return rc;
+  if (s.I % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (w_gate == nullptr || w1 == nullptr || w3 == nullptr || w2 == nullptr ||
+      dw_gate == nullptr || dw1 == nullptr || dw3 == nullptr || dw2 == nullptr ||
+      (s.T > 0 && (x == nullptr || dy == nullptr || dx == nullptr)))
+    return MOE_ERR_INVALID_ARG;
+  if (s.S > 0 && (ws1 == nullptr || ws3 == nullptr || ws2 == nullptr || dws1 == nullptr ||
+                  dws3 == nullptr || dws2 == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, w_gate, w1, w3, w2, ws1, ws3, ws2, dy, dx, dw_gate,
+                        dw1, dw3, dw2, dws1, dws3, dws2};
+  for (const void* q : ptrs)
+    if (!aligned(q, 16)) return MOE_ERR_INVALID_ARG;
+  const moe_train_layout TL = make_train_layout(s);
+  if (workspace == nullptr || workspace_bytes < TL.total || !aligned(workspace, 256))
+    return MOE_ERR_WORKSPACE;
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  const moe_ws_layout& L = TL.fwd;
+
+  BackwardMiscArgs m{};
+  m.x = x;
+  m.dy = dy;
+  m.y_perm = at<uint16_t>(ws, L.y_perm);
+  m.w_gate = w_gate;
+  m.probs = at<float>(ws, L.probs);
+  m.topk_w = at<float>(ws, L.topk_w);
+  m.topk_idx = at<int32_t>(ws, L.topk_idx);
+  m.row_of = at<int32_t>(ws, L.row_of);
+  m.offsets = at<int32_t>(ws, L.offsets);
+  m.token_of_row = at<int32_t>(ws, L.token_of_row);
+  m.dy_perm = at<uint16_t>(ws, TL.dy_perm);
+  m.dw = at<float>(ws, TL.dw);
+  m.dz = at<float>(ws, TL.dz);
+  m.dx_perm = at<float>(ws, TL.dx_perm);
+  m.dx_shared = s.S > 0 ? at<float>(ws, TL.dx_shared) : nullptr;
+  m.dx_router = at<float>(ws, TL.dx_router);
+  m.dwg_partials = at<float>(ws, TL.dwg_partials);
+  m.dw_gate = dw_gate;
+  m.dx = dx;
+  cudaError_t e = bwd_phase(0, st);
+  if (e == cudaSuccess) e = launch_backward_misc_pre(s, m, st);
+  if (e == cudaSuccess) e = bwd_phase(1, st);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+
+  BackwardGemmArgs g{};
+  g.offsets = m.offsets;
+  g.w1 = w1;
+  g.w3 = w3;
+  g.w2 = w2;
+  g.ws1 = ws1;
+  g.ws3 = ws3;
+  g.ws2 = ws2;
+  g.x = x;
+  g.x_perm = at<uint16_t>(ws, L.x_perm);
+  g.h_perm = at<uint16_t>(ws, L.h_perm);
+  g.h_shared = at<uint16_t>(ws, L.h_shared);
+  g.g_perm = at<uint16_t>(ws, TL.g_perm);
+  g.u_perm = at<uint16_t>(ws, TL.u_perm);
+  g.g_shared = at<uint16_t>(ws, TL.g_shared);
+  g.u_shared = at<uint16_t>(ws, TL.u_shared);
+  g.dy = dy;
+  g.dy_perm = m.dy_perm;
+  g.dgu_perm = at<uint16_t>(ws, TL.dgu_perm);
+  g.dgu_shared = at<uint16_t>(ws, TL.dgu_shared);
+  g.dx_perm = at<float>(ws, TL.dx_perm);
+  g.dx_shared = at<float>(ws, TL.dx_shared);
+  g.dw1 = dw1;
+  g.dw3 = dw3;
+  g.dw2 = dw2;
+  g.dws1 = dws1;
+  g.dws3 = dws3;
+  g.dws2 = dws2;
+  e = launch_backward_gemms(s, g, di->num_sms, di->status, g_wait_limit_ns, st,
+                            g_bwd_phase_on ? &g_phase_events[kFwdEvents + 2] : nullptr);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  e = launch_backward_misc_post(s, m, st);
+  if (e == cudaSuccess) e = bwd_phase(6, st);
   return cuda_status(e);
 }
 
@@ -320,15 +498,16 @@ int moe_get_last_device_status(void* stream) {
 
 int moe_set_phase_events(void* const* events, int n) {
   if (events == nullptr || n == 0) {
-    g_phase_on = false;
+    g_phase_on = g_bwd_phase_on = false;
     return MOE_OK;
   }
-  if (n < 6) return MOE_ERR_INVALID_ARG;
-  for (int i = 0; i < 6; ++i) {
+  if (n != kFwdEvents && n != kAllEvents) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
     if (events[i] == nullptr) return MOE_ERR_INVALID_ARG;
     g_phase_events[i] = static_cast<cudaEvent_t>(events[i]);
   }
   g_phase_on = true;
+  g_bwd_phase_on = n == kAllEvents;
   return MOE_OK;
 }
 

@@ -53,11 +53,55 @@ struct GroupedGemmArgs {
   const uint16_t *ws1, *ws3, *ws2;
   uint16_t* h_shared;  // [T, S*I]
   float* y_shared;     // [T, d]
+  // training: pre-activations of the gate/up GEMM (null = not stored)
+  uint16_t* g_perm = nullptr;    // [cap, I]
+  uint16_t* u_perm = nullptr;    // [cap, I]
+  uint16_t* g_shared = nullptr;  // [T, S*I]
+  uint16_t* u_shared = nullptr;  // [T, S*I]
 };
 // `between` (may be null) is recorded on `st` after the gate/up GEMM is launched.
 cudaError_t launch_grouped_gemms(const Shape& s, const GroupedGemmArgs& a, int num_sms,
                                  unsigned int* status, uint64_t wait_limit_ns, cudaStream_t st,
                                  cudaEvent_t between = nullptr);
+
+// ---- backward grouped GEMMs (grouped_gemm_bwd.cu)
+struct BackwardGemmArgs {
+  const int32_t* offsets;
+  const uint16_t *w1, *w3, *w2, *ws1, *ws3, *ws2;
+  const uint16_t *x, *x_perm;                             // forward inputs
+  const uint16_t *h_perm, *h_shared;                      // forward activations
+  const uint16_t *g_perm, *u_perm, *g_shared, *u_shared;  // saved pre-activations
+  const uint16_t *dy, *dy_perm;  // upstream gradient: per token, and w * dy per segment row
+  uint16_t* dgu_perm;    // [cap, 2I]  [dG | dU]
+  uint16_t* dgu_shared;  // [T, 2*S*I]
+  float* dx_perm;        // [cap, d]
+  float* dx_shared;      // [T, d]
+  uint16_t *dw1, *dw3, *dw2, *dws1, *dws3, *dws2;
+};
+// `events` (may be null): 4 events recorded after the dH/SwiGLU dgrad, the dW2
+// wgrad, the dX dgrad and the dW1/dW3 wgrads.
+cudaError_t launch_backward_gemms(const Shape& s, const BackwardGemmArgs& a, int num_sms,
+                                  unsigned int* status, uint64_t wait_ns, cudaStream_t st,
+                                  const cudaEvent_t* events = nullptr);
+
+// ---- backward outside the expert GEMMs (backward.cu)
+struct BackwardMiscArgs {
+  const uint16_t *x, *dy, *y_perm;
+  const float *w_gate, *probs, *topk_w;
+  const int32_t *topk_idx, *row_of, *offsets, *token_of_row;
+  uint16_t* dy_perm;    // [cap, d]
+  float* dw;            // [T, k]
+  float* dz;            // [T, E]
+  const float* dx_perm;    // [cap, d]
+  const float* dx_shared;  // [T, d] or null
+  float* dx_router;     // [T, d]
+  float* dwg_partials;  // [splits, E, d]
+  float* dw_gate;       // [E, d]
+  uint16_t* dx;         // [T, d]
+};
+int dwg_splits(const Shape& s);
+cudaError_t launch_backward_misc_pre(const Shape& s, const BackwardMiscArgs& a, cudaStream_t st);
+cudaError_t launch_backward_misc_post(const Shape& s, const BackwardMiscArgs& a, cudaStream_t st);
 
 // ---- combine (combine.cu)
 cudaError_t launch_combine(const Shape& s, const uint16_t* y_perm, const int32_t* row_of,

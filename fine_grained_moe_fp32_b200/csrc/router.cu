@@ -161,18 +161,31 @@ router_topk_kernel(const float* __restrict__ part, int splits, const float* __re
   const int t = blockIdx.x * kTopkWarps + (threadIdx.x >> 5);
   if (t >= T) return;
 
-  float z[4];
   bool valid[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int e = lane + 32 * i;
-    valid[i] = e < E;
-    double s = 0.0;  // split partials summed in fp64, in split order
-    if (valid[i]) {
-      for (int sp = 0; sp < splits; ++sp) s += (double)part[((size_t)sp * T + t) * E + e];
+  for (int i = 0; i < 4; ++i) valid[i] = lane + 32 * i < E;
+  // split partials summed in fp64 in ascending split order; the loads of 16
+  // splits are issued together so their latencies overlap
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  constexpr int kU = 16;
+  for (int sp0 = 0; sp0 < splits; sp0 += kU) {
+    float v[kU][4];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int sp = min(sp0 + u, splits - 1);  // clamped: every load is in bounds
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        v[u][i] = __ldg(part + ((size_t)sp * T + t) * E + min(lane + 32 * i, E - 1));
     }
-    z[i] = valid[i] ? (float)s : -INFINITY;
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (sp0 + u < splits) acc[i] += (double)v[u][i];
   }
+  float z[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) z[i] = valid[i] ? (float)acc[i] : -INFINITY;
   float m = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));

@@ -27,6 +27,7 @@ EXPORTED = (
     "moe_permute_workspace_size", "moe_permute", "moe_grouped_swiglu", "moe_combine",
     "moe_workspace_size", "moe_forward_layout", "moe_forward", "moe_get_last_device_status",
     "moe_set_wait_limit_ns", "moe_set_phase_events", "moe_route_noalloc",
+    "moe_train_workspace_size", "moe_train_layout_of", "moe_forward_train", "moe_backward",
 )
 
 
@@ -41,6 +42,12 @@ class MoeWsLayout(ctypes.Structure):
         "route_partials", "probs", "topk_idx", "topk_w", "counts", "offsets", "row_of",
         "token_of_row", "permute_scratch", "x_perm", "h_perm", "y_perm", "h_shared",
         "y_shared", "total")]
+
+
+class MoeTrainLayout(ctypes.Structure):
+    _fields_ = [("fwd", MoeWsLayout)] + [(n, ctypes.c_size_t) for n in (
+        "g_perm", "u_perm", "g_shared", "u_shared", "dy_perm", "dw", "dz", "dgu_perm",
+        "dgu_shared", "dx_perm", "dx_shared", "dx_router", "dwg_partials", "total")]
 
 
 class MoEError(RuntimeError):
@@ -78,6 +85,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_set_wait_limit_ns": (I, [ctypes.c_uint64]),
         "moe_set_phase_events": (I, [ctypes.POINTER(ctypes.c_void_p), I]),
         "moe_route_noalloc": (I, [P, V, V, V, V, V, V, V]),
+        "moe_train_workspace_size": (Z, [P]),
+        "moe_train_layout_of": (I, [P, ctypes.POINTER(MoeTrainLayout)]),
+        "moe_forward_train": (I, [P, V, V, V, V, V, V, V, V, V, V, V, Z, V]),
+        "moe_backward": (I, [P, V, V, V, V, V, V, V, V, V, V, Z, V, V, V, V, V, V, V, V, V]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -247,6 +258,44 @@ def forward(dm, x, w_gate, bias, w1, w3, w2, ws1, ws3, ws2, y, workspace, stream
     _check(rc, "moe_forward")
 
 
+def train_workspace_size(dm: MoeDims) -> int:
+    return int(load().moe_train_workspace_size(ctypes.byref(dm)))
+
+
+def train_layout(dm: MoeDims) -> dict:
+    L = MoeTrainLayout()
+    _check(load().moe_train_layout_of(ctypes.byref(dm), ctypes.byref(L)), "moe_train_layout_of")
+    out = {n: getattr(L, n) for n, _ in MoeTrainLayout._fields_ if n != "fwd"}
+    out["fwd"] = {n: getattr(L.fwd, n) for n, _ in MoeWsLayout._fields_}
+    return out
+
+
+def forward_train(dm, x, w_gate, bias, w1, w3, w2, ws1, ws3, ws2, y, workspace, stream=None):
+    _expect(x, torch.bfloat16, (dm.T, dm.d), "x")
+    _expect(y, torch.bfloat16, (dm.T, dm.d), "y")
+    rc = load().moe_forward_train(ctypes.byref(dm), _ptr(x), _ptr(w_gate), _ptr(bias), _ptr(w1),
+                                  _ptr(w3), _ptr(w2), _ptr(ws1), _ptr(ws3), _ptr(ws2), _ptr(y),
+                                  _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "moe_forward_train")
+
+
+def backward(dm, x, w_gate, w1, w3, w2, ws1, ws3, ws2, dy, workspace, grads: dict, stream=None):
+    """grads: dict with preallocated dx, dw_gate, dw1, dw3, dw2, dws1, dws3, dws2."""
+    _expect(dy, torch.bfloat16, (dm.T, dm.d), "dy")
+    _expect(grads["dx"], torch.bfloat16, (dm.T, dm.d), "dx")
+    _expect(grads["dw_gate"], torch.float32, (dm.E, dm.d), "dw_gate")
+    _expect(grads["dw1"], torch.bfloat16, (dm.E, dm.I, dm.d), "dw1")
+    _expect(grads["dw3"], torch.bfloat16, (dm.E, dm.I, dm.d), "dw3")
+    _expect(grads["dw2"], torch.bfloat16, (dm.E, dm.d, dm.I), "dw2")
+    g = grads
+    rc = load().moe_backward(ctypes.byref(dm), _ptr(x), _ptr(w_gate), _ptr(w1), _ptr(w3),
+                             _ptr(w2), _ptr(ws1), _ptr(ws3), _ptr(ws2), _ptr(dy), _ptr(workspace),
+                             workspace.numel(), _ptr(g["dx"]), _ptr(g["dw_gate"]), _ptr(g["dw1"]),
+                             _ptr(g["dw3"]), _ptr(g["dw2"]), _ptr(g.get("dws1")),
+                             _ptr(g.get("dws3")), _ptr(g.get("dws2")), _stream(stream))
+    _check(rc, "moe_backward")
+
+
 def device_status(stream=None) -> int:
     """Synchronise the stream; return and clear the device status word."""
     return int(load().moe_get_last_device_status(_stream(stream)))
@@ -257,12 +306,15 @@ def set_wait_limit_ns(ns: int) -> None:
 
 
 PHASES = ("router", "permute", "gemm_gate_up_swiglu", "gemm_down", "combine")
+BWD_PHASES = ("combine_router_bwd", "dgrad_down_swiglu_bwd", "wgrad_w2", "dgrad_up",
+              "wgrad_w1_w3", "gate_gemms_unpermute")
 
 
 def set_phase_events(events) -> None:
     """Record torch.cuda.Event objects between the kernels of moe_forward
-    (6 events: before the router, then after each of the 5 phases); None
-    turns the hook off."""
+    (6 events: before the router, then after each of the 5 phases) and, with
+    13 events, of moe_backward too (before it, then after each of its 6
+    phases); None turns the hook off."""
     if events is None:
         _check(load().moe_set_phase_events(None, 0), "moe_set_phase_events")
         return
@@ -301,6 +353,36 @@ def workspace_views(dm: MoeDims, ws: torch.Tensor) -> dict:
     }
 
 
+def train_workspace_views(dm: MoeDims, ws: torch.Tensor) -> dict:
+    """Typed views of what moe_forward_train / moe_backward leave in the
+    training workspace (the forward views plus the backward intermediates)."""
+    v = workspace_views(dm, ws)
+    L = train_layout(dm)
+    cap = capacity(dm)
+    T, d, E, k, I, S = dm.T, dm.d, dm.E, dm.k, dm.I, dm.n_shared
+
+    def view(off, n, dtype, shape):
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        return ws[off:off + nbytes].view(dtype).view(*shape)
+
+    bf, f32 = torch.bfloat16, torch.float32
+    v.update({
+        "g_perm": view(L["g_perm"], cap * I, bf, (cap, I)),
+        "u_perm": view(L["u_perm"], cap * I, bf, (cap, I)),
+        "g_shared": view(L["g_shared"], T * S * I, bf, (T, S * I)),
+        "u_shared": view(L["u_shared"], T * S * I, bf, (T, S * I)),
+        "dy_perm": view(L["dy_perm"], cap * d, bf, (cap, d)),
+        "dw": view(L["dw"], T * k, f32, (T, k)),
+        "dz": view(L["dz"], T * E, f32, (T, E)),
+        "dgu_perm": view(L["dgu_perm"], cap * 2 * I, bf, (cap, 2 * I)),
+        "dgu_shared": view(L["dgu_shared"], T * 2 * S * I, bf, (T, 2 * S * I)),
+        "dx_perm": view(L["dx_perm"], cap * d, f32, (cap, d)),
+        "dx_shared": view(L["dx_shared"], T * d, f32, (T, d)),
+        "dx_router": view(L["dx_router"], T * d, f32, (T, d)),
+    })
+    return v
+
+
 class MoELayer:
     """The layer with its weights resident on one device; ``__call__`` runs
     moe_forward into a reusable workspace."""
@@ -327,6 +409,39 @@ class MoELayer:
             self._ws = alloc_workspace(workspace_size(self.dims(T)), self.device)
             self._ws_T = T
         return self._ws
+
+    def train_workspace(self, T: int) -> torch.Tensor:
+        if getattr(self, "_tws", None) is None or self._tws_T != T:
+            self._tws = alloc_workspace(train_workspace_size(self.dims(T)), self.device)
+            self._tws_T = T
+        return self._tws
+
+    def forward_train(self, x: torch.Tensor, y: torch.Tensor | None = None, stream=None):
+        """Forward that keeps what the backward needs in the training workspace."""
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty((T, self.cfg.d), dtype=torch.bfloat16, device=self.device)
+        forward_train(self.dims(T), x, self.w_gate, self.bias, self.w1, self.w3, self.w2,
+                      self.ws1, self.ws3, self.ws2, y, self.train_workspace(T), stream)
+        return y
+
+    def alloc_grads(self, T: int) -> dict:
+        c, dev = self.cfg, self.device
+        bf = dict(dtype=torch.bfloat16, device=dev)
+        return {"dx": torch.empty((T, c.d), **bf),
+                "dw_gate": torch.empty((c.E, c.d), dtype=torch.float32, device=dev),
+                "dw1": torch.empty((c.E, c.I, c.d), **bf), "dw3": torch.empty((c.E, c.I, c.d), **bf),
+                "dw2": torch.empty((c.E, c.d, c.I), **bf),
+                "dws1": torch.empty((c.S, c.I, c.d), **bf), "dws3": torch.empty((c.S, c.I, c.d), **bf),
+                "dws2": torch.empty((c.S, c.d, c.I), **bf)}
+
+    def backward(self, x: torch.Tensor, dy: torch.Tensor, grads: dict | None = None, stream=None):
+        """Gradients after forward_train on the same x (routing held fixed)."""
+        T = x.shape[0]
+        grads = self.alloc_grads(T) if grads is None else grads
+        backward(self.dims(T), x, self.w_gate, self.w1, self.w3, self.w2, self.ws1, self.ws3,
+                 self.ws2, dy, self.train_workspace(T), grads, stream)
+        return grads
 
     def __call__(self, x: torch.Tensor, y: torch.Tensor | None = None, stream=None):
         T = x.shape[0]

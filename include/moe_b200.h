@@ -225,6 +225,60 @@ int moe_forward(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
                 size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Training: moe_forward_train and moe_backward.
+ * Technical Report, Results: the grouped GEMM is measured in the forward and
+ * in the backward pass.
+ *
+ * moe_forward_train is moe_forward that also keeps the gate/up
+ * pre-activations (g = w1 x, u = w3 x, bf16) for the backward.  Its workspace
+ * (moe_train_workspace_size() bytes, 256-byte aligned) starts with the
+ * forward layout (same offsets as moe_forward_layout) and adds the regions
+ * of moe_train_layout.
+ *
+ * moe_backward takes that workspace after moe_forward_train on the same x and
+ * weights, and the upstream gradient dy [T, d] bf16, and writes
+ *   dx [T, d] bf16, dw_gate [E, d] fp32, dw1, dw3 [E, I, d], dw2 [E, d, I],
+ *   dws1, dws3 [S, I, d], dws2 [S, d, I] (bf16; every element is written,
+ *   experts that received no token get zero).
+ * The routing choice of the forward is held fixed; the bias only enters the
+ * selection key and gets no gradient.  Gradients flow through the combine
+ * weights, the renormalisation and the softmax into w_gate and x.  Extra
+ * limit: I % 128 == 0.
+ * ---------------------------------------------------------------------- */
+typedef struct moe_train_layout {
+  moe_ws_layout fwd;    /* the forward intermediates (moe_forward_layout)  */
+  size_t g_perm;        /* bf16 [cap, I]  gate pre-activations             */
+  size_t u_perm;        /* bf16 [cap, I]  up pre-activations               */
+  size_t g_shared;      /* bf16 [T, S*I]                                   */
+  size_t u_shared;      /* bf16 [T, S*I]                                   */
+  size_t dy_perm;       /* bf16 [cap, d]  w * dy per segment row            */
+  size_t dw;            /* fp32 [T, k]    gradient of the combine weights   */
+  size_t dz;            /* fp32 [T, E]    gradient of the gate logits       */
+  size_t dgu_perm;      /* bf16 [cap, 2I] [dG | dU]                         */
+  size_t dgu_shared;    /* bf16 [T, 2*S*I]                                  */
+  size_t dx_perm;       /* fp32 [cap, d]                                    */
+  size_t dx_shared;     /* fp32 [T, d]                                      */
+  size_t dx_router;     /* fp32 [T, d]    dz w_gate                         */
+  size_t dwg_partials;  /* fp32 [splits, E, d]                              */
+  size_t total;         /* = moe_train_workspace_size()                     */
+} moe_train_layout;
+
+size_t moe_train_workspace_size(const moe_dims* dims);
+int moe_train_layout_of(const moe_dims* dims, moe_train_layout* layout);
+int moe_forward_train(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
+                      const float* bias, const moe_bf16* w1, const moe_bf16* w3,
+                      const moe_bf16* w2, const moe_bf16* ws1, const moe_bf16* ws3,
+                      const moe_bf16* ws2, moe_bf16* y, void* workspace,
+                      size_t workspace_bytes, void* stream);
+int moe_backward(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
+                 const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
+                 const moe_bf16* ws1, const moe_bf16* ws3, const moe_bf16* ws2,
+                 const moe_bf16* dy, void* workspace, size_t workspace_bytes,
+                 moe_bf16* dx, float* dw_gate, moe_bf16* dw1, moe_bf16* dw3,
+                 moe_bf16* dw2, moe_bf16* dws1, moe_bf16* dws3, moe_bf16* dws2,
+                 void* stream);
+
+/* ------------------------------------------------------------------------
  * Device status and bounded waits.
  *
  * moe_get_last_device_status: synchronises `stream`, returns the first error
@@ -241,12 +295,16 @@ int moe_get_last_device_status(void* stream);
 int moe_set_wait_limit_ns(uint64_t ns);
 
 /* ------------------------------------------------------------------------
- * moe_set_phase_events -- measurement hook.  With n >= 6 CUDA events
- * (cudaEvent_t handles owned by the caller), every later moe_forward records
- * events[0] before its first kernel and events[1..5] after the router, the
- * permutation, the gate/up GEMM, the down GEMM and the combine, on its stream.
- * n == 0 (or events == NULL) turns the hook off.  Process-wide; the events
- * must outlive every moe_forward issued while they are set.
+ * moe_set_phase_events -- measurement hook.  With n == 6 CUDA events
+ * (cudaEvent_t handles owned by the caller), every later moe_forward /
+ * moe_forward_train records events[0] before its first kernel and
+ * events[1..5] after the router, the permutation, the gate/up GEMM, the down
+ * GEMM and the combine, on its stream.  With n == 13, moe_backward also
+ * records events[6] before its first kernel and events[7..12] after the
+ * combine/router backward, the dH + SwiGLU-backward dgrad, the dW2 wgrad, the
+ * dX dgrad, the dW1/dW3 wgrads and the gate GEMMs + un-permute.  n == 0 (or
+ * events == NULL) turns the hook off.  Process-wide; the events must outlive
+ * every call issued while they are set.
  * ---------------------------------------------------------------------- */
 int moe_set_phase_events(void* const* events, int n);
 

@@ -263,9 +263,10 @@ def silu_grad(g):
     return s * (1.0 + g * (1.0 - s))
 
 
-def swiglu_expert_backward(xr, w1, w3, w2, dout):
+def swiglu_expert_backward(xr, w1, w3, w2, dout, with_pre=False):
     """Gradients of out = W2 (silu(W1 x) * W3 x) for rows xr given dout.
-    Returns dx, dW1, dW3, dW2."""
+    Returns dx, dW1, dW3, dW2 (and dg, du, the gradients at the gate and up
+    pre-activations, when with_pre)."""
     xr, w1, w3, w2, dout = map(_f64, (xr, w1, w3, w2, dout))
     g = xr @ w1.T
     u = xr @ w3.T
@@ -278,10 +279,12 @@ def swiglu_expert_backward(xr, w1, w3, w2, dout):
     dW1 = dg.T @ xr
     dW3 = du.T @ xr
     dx = dg @ w1 + du @ w3
+    if with_pre:
+        return dx, dW1, dW3, dW2, dg, du
     return dx, dW1, dW3, dW2
 
 
-def backward(inp: dict, dy, fwd: dict | None = None) -> dict:
+def backward(inp: dict, dy, fwd: dict | None = None, experts=None) -> dict:
     """Gradients of sum(y * dy) for the whole layer, with the routing choice of
     the forward held fixed.
 
@@ -290,6 +293,10 @@ def backward(inp: dict, dy, fwd: dict | None = None) -> dict:
     softmax:   dz = p * (dp - <p, dp>)  (dp is zero off the chosen experts)
     gate:      dWg = dz^T x,  dx += dz Wg
     experts:   swiglu_expert_backward per segment and for each shared expert
+
+    ``experts`` (optional) limits which routed experts' weight gradients are
+    kept (returned as dicts expert -> array); every expert still contributes
+    to dx.  At full size the dense [E, I, d] float64 gradients would not fit.
     """
     cfg = inp["cfg"]
     k, E = cfg.k, cfg.E
@@ -314,28 +321,41 @@ def backward(inp: dict, dy, fwd: dict | None = None) -> dict:
     x_perm = fwd["x_perm"]
     off = fwd["offsets"]
     dx_perm = np.zeros_like(x_perm)
-    dW1 = np.zeros(inp["w1"].shape)
-    dW3 = np.zeros(inp["w3"].shape)
-    dW2 = np.zeros(inp["w2"].shape)
+    keep = range(E) if experts is None else [int(e) for e in experts]
+    if experts is None:
+        dW1 = np.zeros(inp["w1"].shape)
+        dW3 = np.zeros(inp["w3"].shape)
+        dW2 = np.zeros(inp["w2"].shape)
+    else:
+        dW1 = {e: np.zeros(inp["w1"].shape[1:]) for e in keep}
+        dW3 = {e: np.zeros(inp["w3"].shape[1:]) for e in keep}
+        dW2 = {e: np.zeros(inp["w2"].shape[1:]) for e in keep}
+    I = inp["w1"].shape[1]
+    dgu_perm = np.zeros((len(x_perm), 2 * I))
     for e in range(E):
         a, b = int(off[e]), int(off[e + 1])
         if a == b:
             continue
-        dxe, g1, g3, g2 = swiglu_expert_backward(x_perm[a:b], inp["w1"][e],
-                                                 inp["w3"][e], inp["w2"][e],
-                                                 dy_perm[a:b])
+        dxe, g1, g3, g2, dg, du = swiglu_expert_backward(x_perm[a:b], inp["w1"][e],
+                                                         inp["w3"][e], inp["w2"][e],
+                                                         dy_perm[a:b], with_pre=True)
         dx_perm[a:b] = dxe
-        dW1[e], dW3[e], dW2[e] = g1, g3, g2
+        dgu_perm[a:b, :I], dgu_perm[a:b, I:] = dg, du
+        if e in keep:
+            dW1[e], dW3[e], dW2[e] = g1, g3, g2
     S = inp["ws1"].shape[0]
     dWs1 = np.zeros(inp["ws1"].shape)
     dWs3 = np.zeros(inp["ws3"].shape)
     dWs2 = np.zeros(inp["ws2"].shape)
     dx = np.zeros((T, d))
+    dg_sh, du_sh = [], []
     for s in range(S):
-        dxs, g1, g3, g2 = swiglu_expert_backward(x, inp["ws1"][s], inp["ws3"][s],
-                                                 inp["ws2"][s], dy)
+        dxs, g1, g3, g2, dg, du = swiglu_expert_backward(x, inp["ws1"][s], inp["ws3"][s],
+                                                         inp["ws2"][s], dy, with_pre=True)
         dx += dxs
         dWs1[s], dWs3[s], dWs2[s] = g1, g3, g2
+        dg_sh.append(dg)
+        du_sh.append(du)
     for j in range(k):                       # un-permute: gather-sum
         dx += dx_perm[row_of[:, j]]
     # renormalisation and softmax backward, then the gate projection
@@ -348,6 +368,8 @@ def backward(inp: dict, dy, fwd: dict | None = None) -> dict:
     wg = _f64(inp["w_gate"])
     dWg = dz.T @ x
     dx += dz @ wg
+    dgu_shared = np.concatenate(dg_sh + du_sh, axis=1) if S else np.zeros((T, 0))
     return {"dx": dx, "dw_gate": dWg, "dw1": dW1, "dw3": dW3, "dw2": dW2,
             "dws1": dWs1, "dws3": dWs3, "dws2": dWs2, "dw": dw, "dz": dz,
-            "dy_perm": dy_perm, "dx_perm": dx_perm}
+            "dy_perm": dy_perm, "dx_perm": dx_perm, "dgu_perm": dgu_perm,
+            "dgu_shared": dgu_shared}

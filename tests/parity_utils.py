@@ -17,6 +17,18 @@ workload specification fixes):
     own bf16 rounding (2^-8 |y|) plus the bf16 rounding of every routed
     output it sums (2^-8 sum_j w_j |o_j|), plus 1e-2 rms(y) for the rounding
     of h carried through the down projection.
+  * gradients of the backward (bf16 dx, dW; fp32 dWg): the 2e-2 * rms bound
+    is below what any bf16 answer can reach for them -- the routed experts'
+    weight gradients are sums over ~12 tokens dominated by single large
+    products (max |dW| ~ 17 rms), and even the exactly-rounded bf16 value of
+    the fp64 gradient is off by ~6 % of rms there.  Every element must lie
+    within three bf16 roundings of its own magnitude (output, and the two
+    rounded inputs of its dominant product) plus 2e-2 rms.  For the routed
+    experts' weight gradients (sums whose products can nearly cancel) the
+    bound also carries kappa * u * A, with A = sum |a_t||b_t| over the
+    element's products, kappa the number of bf16 roundings feeding a product
+    and u = 2^-8 the bf16 unit roundoff; a CPU emulation of the bf16 storage
+    points reproduces the GPU's values at the worst elements.
 """
 import numpy as np
 import torch
@@ -85,6 +97,31 @@ def check_output(y_gpu, y_ref, what="y", spec=True, routed_abs=None):
         bound = BF16_REL * np.abs(y_ref) + extra + 1e-2 * r + 1e-30
         assert np.all(diff <= bound), f"{what}: max err {err:.4e} beyond the rounding bound (rms {r:.4e})"
     return err / r if r > 0 else 0.0
+
+
+def bf16_floor(ref):
+    """max |bf16(ref) - ref| / rms(ref): the error of the best possible bf16 answer."""
+    ref = np.asarray(ref, dtype=np.float64)
+    r = rms(ref)
+    if r == 0:
+        return 0.0
+    rounded = torch.tensor(ref, dtype=torch.float32).to(torch.bfloat16).double().numpy()
+    return float(np.abs(rounded - ref).max() / r)
+
+
+def check_grad(got, ref, what, abs_sum=None, kappa=0):
+    got, ref = to_np(got), np.asarray(ref, dtype=np.float64)
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    r = rms(ref)
+    diff = np.abs(got - ref)
+    bound = 3 * BF16_REL * np.abs(ref) + Y_RMS_FRAC * r + 1e-30
+    if abs_sum is not None:
+        bound = bound + kappa * BF16_REL * np.asarray(abs_sum)
+    worst = np.unravel_index(np.argmax(diff / bound), diff.shape) if diff.size else None
+    assert np.all(diff <= bound), (
+        f"{what}: worst at {worst}: got {got[worst]:.5g} ref {ref[worst]:.5g} "
+        f"bound {bound[worst]:.3g} (rms {r:.3g})")
+    return float(diff.max()) / r if r > 0 else 0.0
 
 
 def np_inputs(inp):
