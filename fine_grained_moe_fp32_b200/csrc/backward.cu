@@ -132,83 +132,154 @@ router_bwd_kernel(const float* __restrict__ probs, const int32_t* __restrict__ t
   }
 }
 
-// fp32 GEMM on CUDA cores: C[m, n] (+)= sum_k A(m, k) B(k, n).
+// fp32 GEMM on CUDA cores: C[m, n] = sum_k A(m, k) B(k, n) over one K split.
 //   A(m, k) = a[m * lda + k]  (A_MMAJOR = false)  or  a[k * lda + m]  (true)
-//   B(k, n) = b[k * ldb + n]  (TB = float or bf16 bits)
-// 128 x 128 tile, 16-deep k chunks in smem, 16 x 16 threads of 8 x 8
-// outputs; fp32 chunk sums added into an fp64 running sum.  blockIdx.z is the
-// split of K; each split writes its own partial C slab.
+//   B(k, n) = b[k * ldb + n]  (TB = float, or bf16 bits)
+// 128 x 128 tile, 16-deep k chunks double-buffered in smem with the next
+// chunk prefetched into registers; 16 x 16 threads of 8 x 8 outputs, one fp32
+// running sum each (these gradients are held to bf16-level tolerances; an
+// fp32 sum of K = 8192 terms is good to ~1e-5 relative).  blockIdx.z is the split of K; each split writes
+// its own partial C slab.  Requires lda % 4 == 0 and ldb % 8 == 0.
 constexpr int SB = 128, SK = 16, kSgThreads = 256;
 
 template <bool A_MMAJOR, typename TB>
-__global__ void __launch_bounds__(kSgThreads, 1)
+__global__ void __launch_bounds__(kSgThreads, 2)
 sgemm_kernel(const float* __restrict__ a, int lda, const TB* __restrict__ b, int ldb,
              float* __restrict__ c, int ldc, int64_t c_split_stride, int M, int N, int K,
              int kchunk) {
-  __shared__ __align__(16) float As[SK][SB];
-  __shared__ __align__(16) float Bs[SK][SB];
+  __shared__ __align__(16) float As[2][SK][SB];
+  __shared__ __align__(16) float Bs[2][SK][SB];
   const int tid = threadIdx.x;
   const int m0 = blockIdx.y * SB, n0 = blockIdx.x * SB;
   const int k_begin = blockIdx.z * kchunk;
   const int k_end = min(K, k_begin + kchunk);
+  const int nk = (k_end - k_begin + SK - 1) / SK;
   const int ty = tid >> 4, tx = tid & 15;
-  double acc[8][8];
+
+  float4 ra[2];
+  float4 rb[2];
+  auto load_a = [&](int k0) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (A_MMAJOR) {  // 16 k-rows x 32 float4 along m
+        const int kk = (tid >> 5) + 8 * i, m4 = (tid & 31) * 4;
+        const int gk = k0 + kk, gm = m0 + m4;
+        if (gk < k_end) {
+          const float* src = a + (size_t)gk * lda + gm;
+          if (gm + 3 < M) {
+            v = *reinterpret_cast<const float4*>(src);
+          } else {
+            if (gm < M) v.x = src[0];
+            if (gm + 1 < M) v.y = src[1];
+            if (gm + 2 < M) v.z = src[2];
+          }
+        }
+      } else {  // 128 m-rows x 4 float4 along k
+        const int idx = tid + kSgThreads * i;
+        const int mm = idx >> 2, kq = idx & 3;
+        const int gm = m0 + mm, gk = k0 + kq * 4;
+        if (gm < M) {
+          const float* src = a + (size_t)gm * lda + gk;
+          if (gk + 3 < k_end) {
+            v = *reinterpret_cast<const float4*>(src);
+          } else {
+            if (gk < k_end) v.x = src[0];
+            if (gk + 1 < k_end) v.y = src[1];
+            if (gk + 2 < k_end) v.z = src[2];
+          }
+        }
+      }
+      ra[i] = v;
+    }
+  };
+  auto store_a = [&](int buf) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      if (A_MMAJOR) {
+        const int kk = (tid >> 5) + 8 * i, m4 = (tid & 31) * 4;
+        *reinterpret_cast<float4*>(&As[buf][kk][m4]) = ra[i];
+      } else {
+        const int idx = tid + kSgThreads * i;
+        const int mm = idx >> 2, kq = idx & 3;
+        As[buf][kq * 4 + 0][mm] = ra[i].x;
+        As[buf][kq * 4 + 1][mm] = ra[i].y;
+        As[buf][kq * 4 + 2][mm] = ra[i].z;
+        As[buf][kq * 4 + 3][mm] = ra[i].w;
+      }
+    }
+  };
+  auto load_b = [&](int k0) {
+    if constexpr (sizeof(TB) == 2) {  // 16 k-rows x 16 vectors of 8 bf16
+      const int kk = tid >> 4, n8 = (tid & 15) * 8;
+      const int gk = k0 + kk, gn = n0 + n8;
+      uint4 w = make_uint4(0, 0, 0, 0);
+      if (gk < k_end && gn < N) w = *reinterpret_cast<const uint4*>(b + (size_t)gk * ldb + gn);
+      rb[0] = make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u),
+                          __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u));
+      rb[1] = make_float4(__uint_as_float(w.z << 16), __uint_as_float(w.z & 0xFFFF0000u),
+                          __uint_as_float(w.w << 16), __uint_as_float(w.w & 0xFFFF0000u));
+    } else {  // 16 k-rows x 32 float4
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int kk = (tid >> 5) + 8 * i, n4 = (tid & 31) * 4;
+        const int gk = k0 + kk, gn = n0 + n4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (gk < k_end && gn < N) v = *reinterpret_cast<const float4*>(b + (size_t)gk * ldb + gn);
+        rb[i] = v;
+      }
+    }
+  };
+  auto store_b = [&](int buf) {
+    if constexpr (sizeof(TB) == 2) {
+      const int kk = tid >> 4, n8 = (tid & 15) * 8;
+      *reinterpret_cast<float4*>(&Bs[buf][kk][n8]) = rb[0];
+      *reinterpret_cast<float4*>(&Bs[buf][kk][n8 + 4]) = rb[1];
+    } else {
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int kk = (tid >> 5) + 8 * i, n4 = (tid & 31) * 4;
+        *reinterpret_cast<float4*>(&Bs[buf][kk][n4]) = rb[i];
+      }
+    }
+  };
+
+  float acc[8][8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 
-  for (int k0 = k_begin; k0 < k_end; k0 += SK) {
-    // ---- stage A (128 m x 16 k) into As[k][m]
-    if (A_MMAJOR) {
-      for (int i = tid; i < SK * SB; i += kSgThreads) {
-        const int kk = i / SB, mm = i % SB;
-        const int gm = m0 + mm, gk = k0 + kk;
-        As[kk][mm] = (gm < M && gk < k_end) ? a[(size_t)gk * lda + gm] : 0.f;
-      }
-    } else {
-      for (int i = tid; i < SK * SB; i += kSgThreads) {
-        const int mm = i / SK, kk = i % SK;
-        const int gm = m0 + mm, gk = k0 + kk;
-        As[kk][mm] = (gm < M && gk < k_end) ? a[(size_t)gm * lda + gk] : 0.f;
-      }
+  if (nk > 0) {
+    load_a(k_begin);
+    load_b(k_begin);
+    store_a(0);
+    store_b(0);
+  }
+  __syncthreads();
+  for (int kc = 0; kc < nk; ++kc) {
+    const int buf = kc & 1;
+    if (kc + 1 < nk) {
+      load_a(k_begin + (kc + 1) * SK);
+      load_b(k_begin + (kc + 1) * SK);
     }
-    // ---- stage B (16 k x 128 n) into Bs[k][n]
-    for (int i = tid; i < SK * SB; i += kSgThreads) {
-      const int kk = i / SB, nn = i % SB;
-      const int gk = k0 + kk, gn = n0 + nn;
-      float v = 0.f;
-      if (gk < k_end && gn < N) {
-        if constexpr (sizeof(TB) == 2)
-          v = __uint_as_float((uint32_t)b[(size_t)gk * ldb + gn] << 16);
-        else
-          v = b[(size_t)gk * ldb + gn];
-      }
-      Bs[kk][nn] = v;
-    }
-    __syncthreads();
-    float part[8][8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) part[i][j] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < SK; ++kk) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][64 + ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][64 + tx * 4]);
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
       const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
       const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) part[i][j] = fmaf(av[i], bv[j], part[i][j]);
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[i][j] += (double)part[i][j];
+    if (kc + 1 < nk) {
+      store_a(buf ^ 1);
+      store_b(buf ^ 1);
+    }
     __syncthreads();
   }
   float* cs = c + (size_t)blockIdx.z * c_split_stride;
@@ -217,9 +288,16 @@ sgemm_kernel(const float* __restrict__ a, int lda, const TB* __restrict__ b, int
     const int gm = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
     if (gm >= M) continue;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int gn = n0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + (j - 4));
-      if (gn < N) cs[(size_t)gm * ldc + gn] = (float)acc[i][j];
+    for (int half = 0; half < 2; ++half) {
+      const int gn = n0 + half * 64 + tx * 4;
+      float* dst = cs + (size_t)gm * ldc + gn;
+      if (gn + 3 < N) {
+        *reinterpret_cast<float4*>(dst) = make_float4(acc[i][half * 4], acc[i][half * 4 + 1],
+                                                      acc[i][half * 4 + 2], acc[i][half * 4 + 3]);
+      } else {
+        for (int j = 0; j < 4; ++j)
+          if (gn + j < N) dst[j] = acc[i][half * 4 + j];
+      }
     }
   }
 }
@@ -278,7 +356,7 @@ unpermute_bwd_kernel(const float* __restrict__ dx_shared, const float* __restric
 
 int dwg_splits(const Shape& s) {
   const int tiles = (int)ceil_div(s.d, SB) * (int)ceil_div(s.E, SB);
-  int sp = tiles > 0 ? 148 / tiles : 1;
+  int sp = tiles > 0 ? 296 / tiles : 1;
   sp = sp < 1 ? 1 : sp;
   const int max_sp = s.T / 256 > 0 ? s.T / 256 : 1;
   return sp > max_sp ? max_sp : sp;

@@ -161,10 +161,6 @@ __device__ __forceinline__ Tile decode(const Ctl& c, const BwdParams& p, int til
 
 __device__ __forceinline__ float sigmoid_f(float g) { return 1.0f / (1.0f + __expf(-g)); }
 
-__device__ __forceinline__ float bf16_at(const uint16_t* p, size_t i) {
-  return __uint_as_float((uint32_t)p[i] << 16);
-}
-
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmA_r,
@@ -177,6 +173,9 @@ grouped_gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmA_r,
   extern __shared__ uint8_t dsmem_raw[];
   const uint32_t raw = smem_u32(dsmem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
+  // epilogue staging tile of the SwiGLU backward: g then u, [32][128] bf16 each
+  uint16_t* epi_g = reinterpret_cast<uint16_t*>(dsmem_raw + (sbase - raw) + kStages * kStageBytes);
+  uint16_t* epi_u = epi_g + 32 * 128;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -418,29 +417,54 @@ grouped_gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmA_r,
             }
           }
         } else if (MODE == kDgradDown) {
-          // dH for feature fg and token rows; SwiGLU backward with the stored g, u
-          const int fg = t.mt * 128 + mrow;
+          // SwiGLU backward on a 32-token x 128-feature tile staged in smem:
+          // g and u come in, and dG / dU go out, as coalesced 16-byte rows;
+          // each thread then works on its own feature (TMEM lane) in place.
+          const int f0 = t.mt * 128;
           const uint16_t* gsrc = routed ? p.g_routed : p.g_shared;
           const uint16_t* usrc = routed ? p.u_routed : p.u_shared;
           const int ldgu = routed ? p.ld_gu_routed : p.ld_gu_shared;
           uint16_t* out = static_cast<uint16_t*>(routed ? p.out_routed : p.out_shared);
           const int ldo = routed ? p.ld_routed : p.ld_shared;
           const int ucol = routed ? p.ucol_routed : p.ucol_shared;
+          const int et = threadIdx.x - 64;  // 0..127 over the epilogue warps
+          for (int i = et; i < 32 * 16; i += kEpiThreads) {
+            const int r = i >> 4, cv = i & 15;
+            uint4 gv = make_uint4(0, 0, 0, 0), uv = gv;
+            if (r < nj) {
+              const size_t at = (size_t)(t.row0 + c0 + r) * ldgu + f0 + cv * 8;
+              gv = *reinterpret_cast<const uint4*>(gsrc + at);
+              uv = *reinterpret_cast<const uint4*>(usrc + at);
+            }
+            *reinterpret_cast<uint4*>(epi_g + r * 128 + cv * 8) = gv;
+            *reinterpret_cast<uint4*>(epi_u + r * 128 + cv * 8) = uv;
+          }
+          named_bar_sync(1, kEpiThreads);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (j < nj) {
-              const int row = t.row0 + c0 + j;
               const float dh = __uint_as_float(v[j]);
-              const float g = bf16_at(gsrc, (size_t)row * ldgu + fg);
-              const float u = bf16_at(usrc, (size_t)row * ldgu + fg);
+              const float g = __uint_as_float((uint32_t)epi_g[j * 128 + mrow] << 16);
+              const float u = __uint_as_float((uint32_t)epi_u[j * 128 + mrow] << 16);
               const float sg = sigmoid_f(g);
-              const float silu = g * sg;
               const float dg = dh * u * (sg * (1.0f + g * (1.0f - sg)));
-              const float du = dh * silu;
-              out[(size_t)row * ldo + fg] = __bfloat16_as_ushort(__float2bfloat16_rn(dg));
-              out[(size_t)row * ldo + ucol + fg] = __bfloat16_as_ushort(__float2bfloat16_rn(du));
+              const float du = dh * (g * sg);
+              epi_g[j * 128 + mrow] = __bfloat16_as_ushort(__float2bfloat16_rn(dg));
+              epi_u[j * 128 + mrow] = __bfloat16_as_ushort(__float2bfloat16_rn(du));
             }
           }
+          named_bar_sync(1, kEpiThreads);
+          for (int i = et; i < 32 * 16; i += kEpiThreads) {
+            const int r = i >> 4, cv = i & 15;
+            if (r < nj) {
+              const size_t row = (size_t)(t.row0 + c0 + r) * ldo + f0 + cv * 8;
+              *reinterpret_cast<uint4*>(out + row) =
+                  *reinterpret_cast<const uint4*>(epi_g + r * 128 + cv * 8);
+              *reinterpret_cast<uint4*>(out + row + ucol) =
+                  *reinterpret_cast<const uint4*>(epi_u + r * 128 + cv * 8);
+            }
+          }
+          named_bar_sync(1, kEpiThreads);  // the tile is reused by the next chunk
         } else {
           // dX for feature o and token rows (fp32: the k routed rows of a
           // token are summed later, so they are not rounded to bf16 here)
@@ -498,7 +522,7 @@ bool make_map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, 
 
 template <int MODE>
 cudaError_t launch_bwd(const CUtensorMap* m, const BwdParams& p, int num_sms, cudaStream_t st) {
-  constexpr size_t smem = (size_t)kStages * kStageBytes + 1024;
+  constexpr size_t smem = (size_t)kStages * kStageBytes + 2 * 32 * 128 * 2 + 1024;
   static_assert(smem + sizeof(Ctl) <= 232448, "shared memory budget");
   auto kern = grouped_gemm_bwd_kernel<MODE>;
   cudaError_t err =

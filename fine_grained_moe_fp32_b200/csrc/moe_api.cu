@@ -396,7 +396,7 @@ int moe_backward(const moe_dims* dims, const moe_bf16* x, const float* w_gate, c
   Shape s;
   int rc = check_dims(dims, &s);
   if (rc != MOE_OK) return rc;
-  if (s.I % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s.I % 128 != 0 || s.E % 4 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (w_gate == nullptr || w1 == nullptr || w3 == nullptr || w2 == nullptr ||
       dw_gate == nullptr || dw1 == nullptr || dw3 == nullptr || dw2 == nullptr ||
       (s.T > 0 && (x == nullptr || dy == nullptr || dx == nullptr)))

@@ -243,7 +243,7 @@ int moe_forward(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
  * The routing choice of the forward is held fixed; the bias only enters the
  * selection key and gets no gradient.  Gradients flow through the combine
  * weights, the renormalisation and the softmax into w_gate and x.  Extra
- * limit: I % 128 == 0.
+ * limits: I % 128 == 0 (moe_forward_train too) and E % 4 == 0.
  * ---------------------------------------------------------------------- */
 typedef struct moe_train_layout {
   moe_ws_layout fwd;    /* the forward intermediates (moe_forward_layout)  */
