@@ -469,6 +469,8 @@ cudaError_t launch_grouped_gemms(const Shape& s, const GroupedGemmArgs& a, int n
                       a.ws2 != nullptr && a.h_shared != nullptr && a.y_shared != nullptr &&
                       s.T > 0;
   const bool small = (int64_t)s.T * s.k <= (int64_t)24 * s.E;  // decode-sized segments
+  if (!small && pair_gemms_supported(s))
+    return launch_grouped_gemms_pair(s, a, num_sms, status, wait_limit_ns, st, between);
   const uint32_t boxB = kBoxB;
   CUtensorMap m[6];
   // ---- gate/up GEMM + SwiGLU

@@ -64,6 +64,12 @@ cudaError_t launch_grouped_gemms(const Shape& s, const GroupedGemmArgs& a, int n
                                  unsigned int* status, uint64_t wait_limit_ns, cudaStream_t st,
                                  cudaEvent_t between = nullptr);
 
+// ---- paired-CTA grouped GEMMs for prefill-sized segments (grouped_gemm_pair.cu)
+bool pair_gemms_supported(const Shape& s);
+cudaError_t launch_grouped_gemms_pair(const Shape& s, const GroupedGemmArgs& a, int num_sms,
+                                      unsigned int* status, uint64_t wait_limit_ns,
+                                      cudaStream_t st, cudaEvent_t between);
+
 // ---- backward grouped GEMMs (grouped_gemm_bwd.cu)
 struct BackwardGemmArgs {
   const int32_t* offsets;

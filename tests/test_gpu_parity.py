@@ -160,6 +160,7 @@ GEMM_CASES = [
     ("tiny_align128", CONFIGS[0], None, 128),
     ("small_ragged", small_config(T=333, d=256, E=16, k=4, I=192), None, 16),
     ("decode_full", CONFIGS[1], None, 16),
+    ("pair_prefill_T700", small_config(T=700, d=512, E=16, k=4, I=256), None, 16),
 ]
 
 
@@ -235,6 +236,8 @@ FWD_CASES = [
     ("tiny_align128", CONFIGS[0], None, 128),
     ("small_ragged_T333", small_config(T=333, d=256, E=16, k=4, I=192), None, 16),
     ("single_token", small_config(T=1, d=256, E=16, k=4, I=128), None, 16),
+    ("pair_prefill_T700", small_config(T=700, d=512, E=16, k=4, I=256), None, 16),
+    ("pair_prefill_align128", small_config(T=700, d=512, E=16, k=4, I=256), None, 128),
     ("no_shared", MoEConfig("noshared", T=200, d=256, E=32, k=6, S=0, I=128,
                             bias="uniform0.01"), None, 16),
     ("one_shared_k8", MoEConfig("s1k8", T=130, d=384, E=64, k=8, S=1, I=256,
