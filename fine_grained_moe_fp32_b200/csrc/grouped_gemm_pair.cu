@@ -11,8 +11,11 @@
 //    token rows; the even CTA ("leader") issues tcgen05.mma.cta_group::2,
 //    which reads A and B from both CTAs' shared memory and leaves each CTA's
 //    128 output rows in its own TMEM.  Per SM this halves the token bytes
-//    loaded per flop, so 6 stages of 32 KB fit where the 1-CTA kernel holds 4
-//    of 48 KB -- the 1-CTA kernel is latency-bound on prefill segments.
+//    loaded per flop.  The weights (from HBM) and the token rows (from L2)
+//    have separate smem rings and producers (6 and 7 stages of 16 KB): the
+//    token rows are re-read from L2 by every feature tile of a segment and
+//    their latency, not the HBM weight stream, is what stalls the MMA when
+//    the two share one shallow ring (measured with per-role wait counters).
 //  * Both CTAs' TMA loads complete on the leader's "full" barrier (the
 //    leader arms it with the pair's byte count); the leader's MMA commits
 //    arrive on the "empty" / "tmem full" barriers of both CTAs at once; both
@@ -31,14 +34,19 @@ namespace {
 
 enum PairMode : int { kPairSwiGLU = 0, kPairDown = 1 };
 
-constexpr int kBK = 64;
-constexpr int kBoxB = 32;
-constexpr int kABytes = 128 * 128;          // this CTA's 128 A rows x 64 K (bf16)
+constexpr int kBK = 128;                    // K per stage: two 64-wide swizzle sub-tiles
+constexpr int kSubK = 64;
+constexpr int kBoxB = 128;                  // one TMA box covers this CTA's token rows
+constexpr int kASub = 128 * 128;            // one K sub-tile of this CTA's 128 A rows
+constexpr int kABytes = 2 * kASub;
 constexpr int kNT = 256;                    // tokens per pair tile
-constexpr int kBBytes = (kNT / 2) * 128;    // this CTA's half of the token rows
-constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kStages = 6;
-constexpr int kThreads = 192;
+constexpr int kBSub = (kNT / 2) * 128;     // one K sub-tile of this CTA's half of the tokens
+constexpr int kBBytes = 2 * kBSub;
+// One ring of 64 KB stages (weights 32 KB, tokens 32 KB) filled by two
+// producer threads -- weights and tokens -- that both arm the stage's full
+// barrier; one commit frees a stage after its 8 MMAs.
+constexpr int kStages = 3;
+constexpr int kThreads = 224;               // warp 6 = token producer
 constexpr int kEpiThreads = 128;
 constexpr uint32_t kTmemCols = 2 * kNT;
 constexpr int kMaxGroups = 129;
@@ -128,7 +136,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
   extern __shared__ uint8_t dsmem_raw[];
   const uint32_t raw = smem_u32(dsmem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
-  float* up_buf = reinterpret_cast<float*>(dsmem_raw + (sbase - raw) + kStages * kStageBytes);
+  float* up_buf =
+      reinterpret_cast<float*>(dsmem_raw + (sbase - raw) + kStages * (kABytes + kBBytes));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -182,7 +191,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
     }
     if (lane == 0) {
       for (int s = 0; s < kStages; ++s) {
-        mbar_init(smem_u32(&ctl.full[s]), 1);
+        mbar_init(smem_u32(&ctl.full[s]), 2);  // armed by both producers
         mbar_init(smem_u32(&ctl.empty[s]), 1);
       }
       for (int b = 0; b < 2; ++b) {
@@ -209,11 +218,14 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
   const int pair = (int)cluster_id_x();
   const int npairs = (int)nclusters_x();
 
-  if (warp == 0) {
-    // ================= TMA producer (both CTAs) =================
+  if (warp == 0 || warp == 6) {
+    // ========== TMA producers (both CTAs): warp 0 weights, warp 6 tokens ==========
     if (lane == 0) {
-      const uint64_t pol_a = policy_evict_normal();
-      const uint64_t pol_b = policy_evict_last();
+      const bool wA = warp == 0;
+      const int nst = kStages;
+      uint64_t* fullb = ctl.full;
+      uint64_t* emptyb = ctl.empty;
+      const uint64_t pol = wA ? policy_evict_normal() : policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // leader: stages whose full phase it armed
@@ -226,45 +238,52 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
         const CUtensorMap* tB = routed ? &tmB_r : &tmB_s;
         const int half = t.nmma >> 1;
         const int nbox = (half + kBoxB - 1) / kBoxB;
-        const uint32_t tx_pair = 2u * (uint32_t)(kABytes + nbox * kBoxB * 128);
+        const uint32_t tx_pair = wA ? 2u * kABytes : 2u * 2u * (uint32_t)(nbox * kBoxB * 128);
         const int arow = MODE == kPairSwiGLU
                              ? (routed ? t.g * p.a_rows_group : 0) + t.ft * 128 + (int)rank * 64
                              : (routed ? t.g * p.a_rows_group : 0) + t.ft * 256 + (int)rank * 128;
         const int brow = t.row0 + (int)rank * half;
         for (int kc = 0; kc < t.kit; ++kc) {
           if (paborted(ctl)) { ok = false; break; }
-          if (!mbar_wait_bounded(smem_u32(&ctl.empty[stage]), phase ^ 1u, p.wait_limit_ns)) {
+          if (!mbar_wait_bounded(smem_u32(&emptyb[stage]), phase ^ 1u, p.wait_limit_ns)) {
             precord_timeout(ctl, p);
             ok = false;
             break;
           }
-          const uint32_t fb_local = smem_u32(&ctl.full[stage]);
+          const uint32_t fb_local = smem_u32(&fullb[stage]);
           const uint32_t fb = mapa_shared(fb_local, 0);  // the leader's barrier
           if (leader) {
             mbar_arrive_expect_tx(fb_local, tx_pair);
             armed |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           }
-          const uint32_t sA = sbase + stage * kStageBytes;
-          const uint32_t sB = sA + kABytes;
           const int kk = kc * kBK;
-          if (MODE == kPairSwiGLU) {
-            tma_load_3d_pair(sA, tA, fb, kk, arow, 0, pol_a);
-            tma_load_3d_pair(sA + kABytes / 2, tA2, fb, kk, arow, 0, pol_a);
-          } else {
-            const int plane = kk / p.k_plane;
-            tma_load_3d_pair(sA, tA, fb, kk - plane * p.k_plane, arow, plane, pol_a);
+          const uint32_t sA = sbase + stage * (kABytes + kBBytes);
+          const uint32_t sB = sA + kABytes;
+          for (int j = 0; j < 2; ++j) {  // the two 64-wide K sub-tiles
+            const int kj = kk + j * kSubK;
+            if (wA) {
+              if (MODE == kPairSwiGLU) {
+                tma_load_3d_pair(sA + j * kASub, tA, fb, kj, arow, 0, pol);
+                tma_load_3d_pair(sA + j * kASub + kASub / 2, tA2, fb, kj, arow, 0, pol);
+              } else {
+                const int plane = kj / p.k_plane;
+                tma_load_3d_pair(sA + j * kASub, tA, fb, kj - plane * p.k_plane, arow, plane, pol);
+              }
+            } else {
+              for (int b = 0; b < nbox; ++b)
+                tma_load_3d_pair(sB + j * kBSub + b * kBoxB * 128, tB, fb, kj, brow + b * kBoxB, 0,
+                                 pol);
+            }
           }
-          for (int b = 0; b < nbox; ++b)
-            tma_load_3d_pair(sB + b * kBoxB * 128, tB, fb, kk, brow + b * kBoxB, 0, pol_b);
-          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+          if (++stage == nst) { stage = 0; phase ^= 1u; }
         }
       }
       if (leader) {
         // every phase this CTA armed completes only once both CTAs' bytes land
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < nst; ++s) {
           if (((armed >> s) & 1u) &&
-              !mbar_wait_bounded(smem_u32(&ctl.full[s]), (armed_parity >> s) & 1u, kDrainLimitNs))
+              !mbar_wait_bounded(smem_u32(&fullb[s]), (armed_parity >> s) & 1u, kDrainLimitNs))
             precord_timeout(ctl, p);
         }
       } else if (!ok) {
@@ -301,13 +320,15 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
             break;
           }
           tc_fence_after();
-          const uint32_t sA = sbase + stage * kStageBytes;
+          const uint32_t sA = sbase + stage * (kABytes + kBBytes);
           const uint32_t sB = sA + kABytes;
 #pragma unroll
-          for (int k4 = 0; k4 < kBK / 16; ++k4) {
-            const uint64_t ad = sdesc_kmajor_sw128(sA + k4 * 32);
-            const uint64_t bd = sdesc_kmajor_sw128(sB + k4 * 32);
-            mma_bf16_ss_pair(dt, ad, bd, idesc, (kc | k4) != 0 ? 1u : 0u);
+          for (int k8 = 0; k8 < kBK / 16; ++k8) {
+            const uint32_t off = (k8 >> 2) * kASub + (k8 & 3) * 32;
+            const uint32_t offb = (k8 >> 2) * kBSub + (k8 & 3) * 32;
+            const uint64_t ad = sdesc_kmajor_sw128(sA + off);
+            const uint64_t bd = sdesc_kmajor_sw128(sB + offb);
+            mma_bf16_ss_pair(dt, ad, bd, idesc, (kc | k8) != 0 ? 1u : 0u);
           }
           mma_commit_pair(smem_u32(&ctl.empty[stage]), 0x3);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -321,6 +342,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
     }
   } else {
     // ================= epilogue (warps 2..5, both CTAs) =================
+    // (warps 0, 1 and 6 are handled above)
     const int q = warp & 3;
     const int frow = q * 32 + lane;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&ctl.tempty[0]), 0);
@@ -449,7 +471,7 @@ bool make_map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, 
 
 template <int MODE>
 cudaError_t launch_pair(const CUtensorMap* m, const PairParams& p, int num_sms, cudaStream_t st) {
-  constexpr size_t smem = (size_t)kStages * kStageBytes + 32 * 64 * 4 + 1024;
+  constexpr size_t smem = (size_t)kStages * (kABytes + kBBytes) + 32 * 64 * 4 + 1024;
   static_assert(smem + sizeof(PCtl) <= 232448, "shared memory budget");
   auto kern = grouped_gemm_pair_kernel<MODE>;
   cudaError_t err =
