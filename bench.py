@@ -229,13 +229,16 @@ def oracle_sample(inp, n_tokens, seed=0):
 # ---------------------------------------------------------------- arms
 
 def workload(args):
-    """The configuration, optionally shrunk (fewer experts / tokens with the
-    same per-expert shape) for profiler captures."""
+    """The configuration, optionally shrunk for profiler captures: fewer
+    experts / tokens with the same per-expert shape, or a narrower expert
+    hidden size I (the router's shape T x d x E is then unchanged)."""
     cfg = CONFIGS[args.config]
-    if args.experts or args.tokens:
+    if args.experts or args.tokens or args.inter:
         E = args.experts or cfg.E
         T = args.tokens or cfg.T
-        cfg = dataclasses.replace(cfg, E=E, T=T, name=f"{cfg.name}__E{E}_T{T}")
+        I = args.inter or cfg.I
+        name = f"{cfg.name}__E{E}_T{T}" + (f"_I{I}" if args.inter else "")
+        cfg = dataclasses.replace(cfg, E=E, T=T, I=I, name=name)
     return cfg
 
 
@@ -462,6 +465,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--experts", type=int, default=0, help="shrink E (profiling cases)")
     ap.add_argument("--tokens", type=int, default=0, help="override T (profiling cases)")
+    ap.add_argument("--inter", type=int, default=0, help="override I (profiling cases)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -17,6 +17,7 @@ namespace {
 constexpr int BT = kRouterBT;  // tokens per tile
 constexpr int BE = 128;        // experts per tile (all of them; E <= 128)
 constexpr int BK = kRouterBK;  // k-chunk in shared memory
+constexpr int kFold = 4;      // staged chunks summed in fp32 before each fp64 add
 constexpr int kThreads = 256;
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {
@@ -25,11 +26,13 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {
 
 // 256 threads as a 16 x 16 grid; thread (ty, tx) owns tokens
 // {ty*4 .. ty*4+3, 64+ty*4 .. 64+ty*4+3} and experts {tx*4 .., 64+tx*4 ..}.
-// Accumulation is two-level: the products are fp32 FMAs and the BK products
-// of one staged chunk are summed from zero in fp32; the running sum across
-// chunks is carried in fp64 (one add per BK FMAs).  A single fp32 running sum
-// over k = 5120 terms loses ~1e-5 relative in the softmax probabilities when
-// one term is large (e.g. a logit offset); this keeps it near 1e-7.
+// Accumulation is two-level: the products are fp32 FMAs and the kFold*BK
+// products of kFold staged chunks are summed from zero in fp32; the running
+// sum across those groups is carried in fp64 (one conversion and add per
+// kFold*BK FMAs, so the slow float->double conversions stay a small share of
+// the issue slots).  A single fp32 running sum over k = 5120 terms loses
+// ~1e-5 relative in the softmax probabilities when one term is large (e.g. a
+// logit offset); with 64-term fp32 groups the error stays near 2e-6.
 __global__ void __launch_bounds__(kThreads, 1)
 router_gemm_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wg,
                    float* __restrict__ part, int T, int d, int E, int kchunk) {
@@ -90,14 +93,14 @@ router_gemm_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wg,
     sstore(0);
   }
   __syncthreads();
+  float part_acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) part_acc[i][j] = 0.f;
   for (int kc = 0; kc < nk; ++kc) {
     const int buf = kc & 1;
     if (kc + 1 < nk) gload(kc + 1);
-    float part_acc[8][8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) part_acc[i][j] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < BK; ++kk) {
       const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][kk][ty * 4]);
@@ -111,10 +114,15 @@ router_gemm_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wg,
 #pragma unroll
         for (int j = 0; j < 8; ++j) part_acc[i][j] = fmaf(a[i], b[j], part_acc[i][j]);
     }
+    if ((kc % kFold) == kFold - 1 || kc + 1 == nk) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc[i][j] += (double)part_acc[i][j];
+        for (int j = 0; j < 8; ++j) {
+          acc[i][j] += (double)part_acc[i][j];
+          part_acc[i][j] = 0.f;
+        }
+    }
     if (kc + 1 < nk) sstore(buf ^ 1);
     __syncthreads();
   }
@@ -249,15 +257,31 @@ struct SplitPlan {
   int kchunk;
 };
 
+// Split of K: one CTA per SM runs at a time, so pick the split count whose
+// CTA count wastes the least of the last wave (waves / splits smallest),
+// preferring fewer splits on near-ties, within a cap on the partial-logit
+// buffer (16 MiB, or one split per tile if even that exceeds it).
 SplitPlan plan_splits(const Shape& s, int num_sms) {
   const int tiles = (int)ceil_div(s.T, BT);
-  const int max_splits = s.d / (BK * 4) > 0 ? s.d / (BK * 4) : 1;
-  int splits = tiles > 0 ? num_sms / tiles : 1;
-  if (splits < 1) splits = 1;
-  if (splits > max_splits) splits = max_splits;
-  const int kchunk = (int)round_up(ceil_div(s.d, splits), BK);
-  splits = (int)ceil_div(s.d, kchunk);
-  return {splits, kchunk};
+  int max_splits = s.d / (BK * 4) > 0 ? s.d / (BK * 4) : 1;
+  const int64_t per_split = (int64_t)s.T * s.E * (int64_t)sizeof(float);
+  const int64_t cap_bytes = int64_t(16) << 20;
+  if (per_split > 0 && max_splits > cap_bytes / per_split)
+    max_splits = (int)(cap_bytes / per_split) > 0 ? (int)(cap_bytes / per_split) : 1;
+  int best = 1;
+  double best_cost = 1e30;
+  for (int sp = 1; sp <= max_splits && tiles > 0; ++sp) {
+    const int kchunk = (int)round_up(ceil_div(s.d, sp), BK);
+    const int real = (int)ceil_div(s.d, kchunk);
+    const double waves = (double)ceil_div((int64_t)tiles * real, num_sms);
+    const double cost = waves * kchunk;  // time ~ waves x work per CTA
+    if (cost < best_cost * 0.98) {
+      best_cost = cost;
+      best = real;
+    }
+  }
+  const int kchunk = (int)round_up(ceil_div(s.d, best), BK);
+  return {(int)ceil_div(s.d, kchunk), kchunk};
 }
 
 }  // namespace
