@@ -373,3 +373,61 @@ def backward(inp: dict, dy, fwd: dict | None = None, experts=None) -> dict:
             "dws1": dWs1, "dws3": dWs3, "dws2": dWs2, "dw": dw, "dz": dz,
             "dy_perm": dy_perm, "dx_perm": dx_perm, "dgu_perm": dgu_perm,
             "dgu_shared": dgu_shared}
+
+
+# --------------------------------------------------------------------------
+# Load balancing, training side (Technical Report, Method: the DeepSeek
+# auxiliary-loss-free bias update, complemented by a sequence-wise balance
+# loss against extreme imbalance inside one sequence).  The pages name both
+# mechanisms but give no formula; the forms below are the published DeepSeek
+# ones the report points to (the reading is listed in the design notes).
+# --------------------------------------------------------------------------
+
+def balance_stats(probs, idx, E: int, k: int, seq_len: int, alpha: float) -> dict:
+    """Sequence-wise balance statistics and loss.
+
+    The T tokens are T / seq_len consecutive sequences of seq_len tokens.  For
+    sequence s and expert e:
+
+      f[s, e] = E / (k * seq_len) * (number of (token, slot) pairs of s routed to e)
+      P[s, e] = (1 / seq_len) * sum over the tokens t of s of probs[t, e]
+
+    (softmax probabilities already sum to 1 per token, so they are their own
+    normalised affinities), and
+
+      loss = alpha / n_seq * sum_s sum_e f[s, e] * P[s, e]
+
+    i.e. the mean over sequences of alpha * sum_e f * P.  Returns f, P
+    [n_seq, E], the per-sequence selection counts and the loss.
+    """
+    p = _f64(probs)
+    idx = np.asarray(idx, dtype=np.int64)
+    T = idx.shape[0]
+    assert seq_len > 0 and T % seq_len == 0, "T must be a whole number of sequences"
+    n_seq = T // seq_len
+    f = np.zeros((n_seq, E))
+    P = np.zeros((n_seq, E))
+    counts = np.zeros((n_seq, E), dtype=np.int64)
+    for s in range(n_seq):
+        t0, t1 = s * seq_len, (s + 1) * seq_len
+        for t in range(t0, t1):
+            for j in range(k):
+                counts[s, idx[t, j]] += 1
+        f[s] = E * counts[s] / (k * seq_len)
+        P[s] = p[t0:t1].sum(axis=0) / seq_len
+    loss = alpha * float(np.sum(f * P)) / n_seq if n_seq else 0.0
+    return {"f": f, "P": P, "counts": counts, "loss": loss}
+
+
+def bias_update(bias, counts, gamma: float, T: int, k: int) -> np.ndarray:
+    """Auxiliary-loss-free bias step: an expert that received more than the
+    mean load T*k/E of the batch has its bias lowered by gamma, one that
+    received less has it raised by gamma, one exactly at the mean keeps it.
+    ``counts`` are the batch's per-expert pair counts (summed over all
+    data-parallel replicas when there are several)."""
+    b = _f64(bias)
+    c = np.asarray(counts, dtype=np.int64)
+    E = b.shape[0]
+    excess = E * c - T * k                 # E * (count - mean), exact integers
+    step = -np.sign(excess).astype(np.float64)
+    return np.where(step == 0, b, b + gamma * step)

@@ -370,3 +370,95 @@ def test_backward_bias_gets_no_gradient():
     y1 = O.forward(inp)
     assert (y0["idx"] == y1["idx"]).all()
     assert np.sum(y0["y"] * dy) == np.sum(y1["y"] * dy)
+
+
+# ------------------------------------------------------------------ load balancing
+
+def test_balance_hand_example():
+    """Worked example with exact fractions (golden/balance_hand_example.json)."""
+    with open(os.path.join(GOLDEN, "balance_hand_example.json")) as f:
+        g = json.load(f)
+    probs = np.array(_val(g["probs"]))
+    idx = np.array(g["idx"])
+    r = O.balance_stats(probs, idx, g["E"], g["k"], g["seq_len"], _val(g["alpha"]))
+    np.testing.assert_array_equal(r["counts"], g["counts"])
+    np.testing.assert_allclose(r["f"], _val(g["f"]), rtol=1e-15, atol=0)
+    np.testing.assert_allclose(r["P"], _val(g["P"]), rtol=1e-15, atol=0)
+    np.testing.assert_allclose((r["f"] * r["P"]).sum(1), _val(g["sum_fP"]), rtol=1e-15)
+    assert r["loss"] == pytest.approx(_val(g["loss"]), rel=1e-15)
+    nb = O.bias_update(_val(g["bias"]), g["batch_counts"], _val(g["gamma"]), T=len(idx), k=g["k"])
+    np.testing.assert_array_equal(nb, _val(g["bias_next"]))
+
+
+def _balanced_seq(E, k, L):
+    """Every expert gets exactly k*L/E pairs; uniform probabilities."""
+    idx = np.array([[(k * t + j) % E for j in range(k)] for t in range(L)])
+    return np.full((L, E), 1.0 / E), idx
+
+
+def _collapsed_seq(E, k, L):
+    """Every token picks experts 0..k-1 and puts all its mass on them."""
+    p = np.zeros((L, E))
+    p[:, :k] = 1.0 / k
+    return p, np.tile(np.arange(k), (L, 1))
+
+
+def test_balance_closed_forms():
+    """Perfect balance gives f = 1, P = 1/E and loss = alpha; full collapse
+    onto k experts gives f = E/k there, P = 1/k and loss = alpha * E / k; two
+    such sequences give the mean of the two."""
+    E, k, L, alpha = 8, 2, 16, 0.3
+    pb, ib = _balanced_seq(E, k, L)
+    r = O.balance_stats(pb, ib, E, k, L, alpha)
+    np.testing.assert_allclose(r["f"], 1.0, rtol=1e-15)
+    np.testing.assert_allclose(r["P"], 1.0 / E, rtol=1e-15)
+    assert r["loss"] == pytest.approx(alpha, rel=1e-14)
+    pc, ic = _collapsed_seq(E, k, L)
+    r = O.balance_stats(pc, ic, E, k, L, alpha)
+    np.testing.assert_allclose(r["f"][0, :k], E / k, rtol=1e-15)
+    assert not r["f"][0, k:].any() and not r["P"][0, k:].any()
+    assert r["loss"] == pytest.approx(alpha * E / k, rel=1e-14)
+    r = O.balance_stats(np.concatenate([pb, pc]), np.concatenate([ib, ic]), E, k, L, alpha)
+    assert r["loss"] == pytest.approx(alpha * (1 + E / k) / 2, rel=1e-14)
+
+
+def test_balance_invariants_random_routing():
+    """On a random softmax / top-k routing: sum_e f = E and sum_e P = 1 per
+    sequence; the loss does not change when tokens are reordered inside a
+    sequence or when the experts are relabelled (probabilities and ids
+    permuted together), and it does change when only the ids are shuffled."""
+    rng = np.random.default_rng(5)
+    E, k, L, n = 16, 4, 24, 3
+    p = O.softmax(rng.normal(size=(n * L, E)) * 2)
+    idx = np.argsort(-p - rng.uniform(0, 0.05, size=p.shape), axis=1)[:, :k]
+    r = O.balance_stats(p, idx, E, k, L, 1.0)
+    np.testing.assert_allclose(r["f"].sum(1), E, rtol=1e-14)
+    np.testing.assert_allclose(r["P"].sum(1), 1.0, rtol=1e-14)
+    assert r["counts"].sum() == n * L * k
+    perm_t = np.concatenate([s * L + rng.permutation(L) for s in range(n)])
+    r2 = O.balance_stats(p[perm_t], idx[perm_t], E, k, L, 1.0)
+    assert r2["loss"] == pytest.approx(r["loss"], rel=1e-13)
+    relabel = rng.permutation(E)            # expert e becomes relabel[e]
+    p3 = np.empty_like(p)
+    p3[:, relabel] = p
+    r3 = O.balance_stats(p3, relabel[idx], E, k, L, 1.0)
+    assert r3["loss"] == pytest.approx(r["loss"], rel=1e-13)
+    np.testing.assert_allclose(r3["f"][:, relabel], r["f"], rtol=1e-15)
+    r4 = O.balance_stats(p, (idx + 1) % E, E, k, L, 1.0)
+    assert abs(r4["loss"] - r["loss"]) > 1e-3 * r["loss"]
+
+
+def test_bias_update_direction_and_fixed_point():
+    """Overloaded experts move down by gamma, underloaded up by gamma, experts
+    exactly at the mean load keep their bias bit for bit (also -0.0); a batch
+    with every expert at the mean is a fixed point."""
+    T, k, E, gamma = 32, 4, 8, 1e-3
+    mean = T * k // E
+    counts = np.array([mean + 3, mean - 1, mean, mean, mean + 1, mean - 2, mean, mean - 1])
+    assert counts.sum() == T * k
+    bias = np.array([0.5, -0.25, -0.0, 1e-3, 0.0, 0.0, 2.0, -1.0])
+    nb = O.bias_update(bias, counts, gamma, T, k)
+    np.testing.assert_array_equal(np.sign(nb - bias), [-1, 1, 0, 0, -1, 1, 0, 1])
+    np.testing.assert_allclose(np.abs(nb - bias)[nb != bias], gamma, rtol=1e-12)
+    assert np.signbit(nb[2])
+    np.testing.assert_array_equal(O.bias_update(bias, np.full(E, mean), gamma, T, k), bias)
