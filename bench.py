@@ -20,6 +20,7 @@ from __future__ import annotations
 import argparse
 import dataclasses
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -39,6 +40,13 @@ METRIC = "MoE-layer tokens/s (bf16, d=5120, 128E top-6 + 2 shared) and % of roof
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNELS_PER_STEP = 9  # router gemm + top-k, 4 permutation kernels, 2 grouped GEMMs, combine
 BWD_KERNELS = 12      # combine/router bwd (3), 5 grouped GEMMs, 2 gate GEMMs + split sum, un-permute
+BALANCE_KERNELS = 4   # balance partial sums, per-sequence f/P, loss, bias step
+# training-side balancing of the fwd+bwd step: sequences of the 8K pretraining
+# context (Technical Report, Results: 8K extended to 32K later); the loss
+# coefficient and the bias step size are not on the pages (DeepSeek-V3 values)
+BALANCE_SEQ = 8192
+BALANCE_ALPHA = 1e-4
+BALANCE_GAMMA = 1e-3
 
 
 # ---------------------------------------------------------------- helpers
@@ -207,9 +215,9 @@ def cpu_threads():
 
 def oracle_sample(inp, n_tokens, seed=0):
     """Time the fp64 oracle on a seeded sample of the batch's tokens: the
-    forward (per-token path), or for a training workload the forward and the
-    backward of the sampled tokens (input gradients, router and all experts;
-    weight gradients not kept)."""
+    forward (per-token path), or for a training workload the forward, the
+    backward (input gradients, router and all experts; weight gradients not
+    kept), the balance statistics and the bias step of the sampled tokens."""
     from oracle import moe_oracle as O
     host = {k: (v.detach().cpu() if torch.is_tensor(v) else v) for k, v in inp.items()}
     rng = np.random.default_rng(seed)
@@ -221,6 +229,10 @@ def oracle_sample(inp, n_tokens, seed=0):
         sub["x"], sub["dy"], sub["T"] = host["x"][idx], host["dy"][idx], len(toks)
         f = O.forward(sub)
         O.backward(sub, sub["dy"], f, experts=[])
+        cfg = inp["cfg"]
+        O.balance_stats(f["probs"], f["idx"], cfg.E, cfg.k, len(toks), BALANCE_ALPHA)
+        O.bias_update(host["bias"], np.bincount(f["idx"].ravel(), minlength=cfg.E),
+                      BALANCE_GAMMA, len(toks), cfg.k)
     else:
         O.forward_tokens(host, toks)
     return len(toks), time.perf_counter() - t0
@@ -302,12 +314,23 @@ def run_ours(args):
     if train:
         dy = inp["dy"]
         grads = layer.alloc_grads(T)
+        seq_len = math.gcd(T, BALANCE_SEQ)
+        f32 = dict(dtype=torch.float32, device=dev)
+        bal = {"f": torch.empty((T // seq_len, cfg.E), **f32),
+               "P": torch.empty((T // seq_len, cfg.E), **f32), "loss": torch.empty(1, **f32)}
+        bias_next = torch.empty_like(layer.bias)
 
-        def step(xin, yout):
+        def step(xin, yout, evs=None):
             layer.forward_train(xin, yout)
             layer.backward(xin, dy, grads)
+            if evs is not None:
+                evs[0].record(stream)
+            layer.balance_stats(T, seq_len, BALANCE_ALPHA, out=bal)
+            layer.bias_step(T, BALANCE_GAMMA, out=bias_next)
+            if evs is not None:
+                evs[1].record(stream)
     else:
-        def step(xin, yout):
+        def step(xin, yout, evs=None):
             layer(xin, yout)
     n_events = 13 if train else 6
     phase_names = M.PHASES + (M.BWD_PHASES if train else ())
@@ -334,9 +357,11 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     t0 = time.time()
     start.record(stream)
+    bal_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+              for _ in range(args.steps)] if train else [None] * args.steps
     for s in range(args.steps):
         M.set_phase_events(ev[s])
-        step(x, y)
+        step(x, y, bal_ev[s])
     end.record(stream)
     torch.cuda.synchronize(dev)
     t1 = time.time()
@@ -357,6 +382,9 @@ def run_ours(args):
     for i, name in enumerate(M.BWD_PHASES if train else ()):
         phase_ms[name] = statistics.mean(ev[s][6 + i].elapsed_time(ev[s][7 + i])
                                          for s in range(args.steps))
+    if train:
+        phase_ms["balance_stats_bias_step"] = statistics.mean(
+            bal_ev[s][0].elapsed_time(bal_ev[s][1]) for s in range(args.steps))
 
     # ---- end to end through the public API: pinned host x -> y on host
     x_host = x.cpu().pin_memory()
@@ -433,10 +461,12 @@ def run_ours(args):
         "e2e": {"value": e2e_value, "unit": "tokens/s",
                 "h2d_bytes_per_step": T * cfg.d * 2 * (2 if train else 1),
                 "d2h_bytes_per_step": T * cfg.d * 2},
-        "gpu_launches": (KERNELS_PER_STEP + (BWD_KERNELS if train else 0)) * args.steps,
+        "gpu_launches": (KERNELS_PER_STEP + (BWD_KERNELS + BALANCE_KERNELS if train else 0))
+        * args.steps,
     }
     if train:
-        line["config"]["step"] = "forward (training, keeps g/u) + backward"
+        line["config"]["step"] = ("forward (training, keeps g/u) + backward + sequence-wise "
+                                  f"balance statistics (seq_len {seq_len}) + bias step")
         line["train_tflop_per_step"] = sum(train_gemm_flops(cfg, T).values()) / 1e12
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n, dt = oracle_sample(inp, args.cpu_tokens)

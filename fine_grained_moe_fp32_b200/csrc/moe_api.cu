@@ -478,6 +478,40 @@ int moe_backward(const moe_dims* dims, const moe_bf16* x, const float* w_gate, c
   return cuda_status(e);
 }
 
+size_t moe_balance_workspace_size(const moe_dims* dims, int seq_len) {
+  Shape s;
+  if (check_dims(dims, &s) != MOE_OK || seq_len <= 0 || s.T % seq_len != 0) return 0;
+  return balance_workspace_bytes(s, seq_len);
+}
+
+int moe_balance_stats(const moe_dims* dims, int seq_len, const float* probs,
+                      const int32_t* topk_idx, float alpha, float* f, float* P, float* loss,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != MOE_OK) return rc;
+  if (seq_len <= 0 || s.T % seq_len != 0 || loss == nullptr) return MOE_ERR_INVALID_ARG;
+  if (s.T > 0 && (probs == nullptr || topk_idx == nullptr || f == nullptr || P == nullptr ||
+                  workspace == nullptr || !aligned(workspace, 256)))
+    return MOE_ERR_INVALID_ARG;
+  if (s.T > 0 && workspace_bytes < balance_workspace_bytes(s, seq_len)) return MOE_ERR_WORKSPACE;
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return MOE_ERR_CUDA;
+  return cuda_status(launch_balance_stats(s, seq_len, probs, topk_idx, alpha, f, P, loss,
+                                          workspace, di->status,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int moe_bias_update(const moe_dims* dims, const int32_t* counts, float gamma,
+                    const float* bias_in, float* bias_out, void* stream) {
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != MOE_OK) return rc;
+  if (counts == nullptr || bias_in == nullptr || bias_out == nullptr) return MOE_ERR_INVALID_ARG;
+  return cuda_status(
+      launch_bias_update(s, counts, gamma, bias_in, bias_out, static_cast<cudaStream_t>(stream)));
+}
+
 int moe_get_last_device_status(void* stream) {
   const DeviceInfo* di = device_info();
   if (di == nullptr) return MOE_ERR_CUDA;

@@ -109,6 +109,15 @@ int dwg_splits(const Shape& s);
 cudaError_t launch_backward_misc_pre(const Shape& s, const BackwardMiscArgs& a, cudaStream_t st);
 cudaError_t launch_backward_misc_post(const Shape& s, const BackwardMiscArgs& a, cudaStream_t st);
 
+// ---- load balancing, training side (balance.cu)
+size_t balance_workspace_bytes(const Shape& s, int seq_len);
+cudaError_t launch_balance_stats(const Shape& s, int seq_len, const float* probs,
+                                 const int32_t* topk_idx, float alpha, float* f, float* P,
+                                 float* loss, void* workspace, unsigned int* status,
+                                 cudaStream_t st);
+cudaError_t launch_bias_update(const Shape& s, const int32_t* counts, float gamma,
+                               const float* bias_in, float* bias_out, cudaStream_t st);
+
 // ---- combine (combine.cu)
 cudaError_t launch_combine(const Shape& s, const uint16_t* y_perm, const int32_t* row_of,
                            const float* topk_w, const float* y_shared, uint16_t* y,

@@ -28,6 +28,7 @@ EXPORTED = (
     "moe_workspace_size", "moe_forward_layout", "moe_forward", "moe_get_last_device_status",
     "moe_set_wait_limit_ns", "moe_set_phase_events", "moe_route_noalloc",
     "moe_train_workspace_size", "moe_train_layout_of", "moe_forward_train", "moe_backward",
+    "moe_balance_workspace_size", "moe_balance_stats", "moe_bias_update",
 )
 
 
@@ -89,6 +90,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_train_layout_of": (I, [P, ctypes.POINTER(MoeTrainLayout)]),
         "moe_forward_train": (I, [P, V, V, V, V, V, V, V, V, V, V, V, Z, V]),
         "moe_backward": (I, [P, V, V, V, V, V, V, V, V, V, V, Z, V, V, V, V, V, V, V, V, V]),
+        "moe_balance_workspace_size": (Z, [P, I]),
+        "moe_balance_stats": (I, [P, I, V, V, ctypes.c_float, V, V, V, V, Z, V]),
+        "moe_bias_update": (I, [P, V, ctypes.c_float, V, V, V]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -296,6 +300,34 @@ def backward(dm, x, w_gate, w1, w3, w2, ws1, ws3, ws2, dy, workspace, grads: dic
     _check(rc, "moe_backward")
 
 
+def balance_workspace_size(dm: MoeDims, seq_len: int) -> int:
+    return int(load().moe_balance_workspace_size(ctypes.byref(dm), int(seq_len)))
+
+
+def balance_stats(dm, seq_len, probs, topk_idx, alpha, f, P, loss, workspace, stream=None):
+    """Sequence-wise balance statistics f, P [T/seq_len, E] and the loss [1]."""
+    n_seq = dm.T // seq_len if seq_len > 0 else 0
+    _expect(probs, torch.float32, (dm.T, dm.E), "probs")
+    _expect(topk_idx, torch.int32, (dm.T, dm.k), "topk_idx")
+    _expect(f, torch.float32, (n_seq, dm.E), "f")
+    _expect(P, torch.float32, (n_seq, dm.E), "P")
+    _expect(loss, torch.float32, (1,), "loss")
+    rc = load().moe_balance_stats(ctypes.byref(dm), int(seq_len), _ptr(probs), _ptr(topk_idx),
+                                  float(alpha), _ptr(f), _ptr(P), _ptr(loss), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "moe_balance_stats")
+
+
+def bias_update(dm, counts, gamma, bias_in, bias_out, stream=None):
+    """One auxiliary-loss-free bias step (bias_out may be bias_in)."""
+    _expect(counts, torch.int32, (dm.E,), "counts")
+    _expect(bias_in, torch.float32, (dm.E,), "bias_in")
+    _expect(bias_out, torch.float32, (dm.E,), "bias_out")
+    rc = load().moe_bias_update(ctypes.byref(dm), _ptr(counts), float(gamma), _ptr(bias_in),
+                                _ptr(bias_out), _stream(stream))
+    _check(rc, "moe_bias_update")
+
+
 def device_status(stream=None) -> int:
     """Synchronise the stream; return and clear the device status word."""
     return int(load().moe_get_last_device_status(_stream(stream)))
@@ -383,6 +415,19 @@ def train_workspace_views(dm: MoeDims, ws: torch.Tensor) -> dict:
     return v
 
 
+def global_loads(counts: torch.Tensor, T: int, group=None):
+    """Per-expert loads and token count of the whole data-parallel batch: the
+    sum over the ranks of ``group`` (unchanged when there is no group)."""
+    if group is None:
+        return counts, int(T)
+    import torch.distributed as dist
+    c = counts.clone()
+    n = torch.tensor([int(T)], dtype=torch.int64, device=counts.device)
+    dist.all_reduce(c, group=group)
+    dist.all_reduce(n, group=group)
+    return c, int(n.item())
+
+
 class MoELayer:
     """The layer with its weights resident on one device; ``__call__`` runs
     moe_forward into a reusable workspace."""
@@ -442,6 +487,42 @@ class MoELayer:
         backward(self.dims(T), x, self.w_gate, self.w1, self.w3, self.w2, self.ws1, self.ws3,
                  self.ws2, dy, self.train_workspace(T), grads, stream)
         return grads
+
+    def _routing_views(self, T: int, train: bool) -> dict:
+        ws = self.train_workspace(T) if train else self.workspace(T)
+        return workspace_views(self.dims(T), ws)
+
+    def balance_stats(self, T: int, seq_len: int, alpha: float, train: bool = True,
+                      out: dict | None = None, stream=None) -> dict:
+        """Sequence-wise balance statistics of the last forward over T tokens
+        (forward_train when ``train``, else __call__): f, P and the loss."""
+        dm = self.dims(T)
+        v = self._routing_views(T, train)
+        n_seq = T // seq_len
+        if out is None:
+            f32 = dict(dtype=torch.float32, device=self.device)
+            out = {"f": torch.empty((n_seq, self.cfg.E), **f32),
+                   "P": torch.empty((n_seq, self.cfg.E), **f32),
+                   "loss": torch.empty(1, **f32)}
+        key = (T, seq_len)
+        if getattr(self, "_bal_key", None) != key:
+            self._bal_ws = alloc_workspace(balance_workspace_size(dm, seq_len), self.device)
+            self._bal_key = key
+        balance_stats(dm, seq_len, v["probs"], v["topk_idx"], alpha, out["f"], out["P"],
+                      out["loss"], self._bal_ws, stream)
+        return out
+
+    def bias_step(self, T: int, gamma: float, out: torch.Tensor | None = None, train: bool = True,
+                  group=None, stream=None) -> torch.Tensor:
+        """One auxiliary-loss-free bias step from the expert counts of the last
+        forward over T tokens; writes into ``out`` (default: the layer's bias).
+        With a torch.distributed ``group`` of data-parallel replicas the loads
+        and token counts are summed over the group first, so every replica
+        takes the same step as one replica holding the whole batch would."""
+        out = self.bias if out is None else out
+        counts, T_all = global_loads(self._routing_views(T, train)["counts"], T, group)
+        bias_update(self.dims(T_all), counts, gamma, self.bias, out, stream)
+        return out
 
     def __call__(self, x: torch.Tensor, y: torch.Tensor | None = None, stream=None):
         T = x.shape[0]

@@ -279,6 +279,51 @@ int moe_backward(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
                  void* stream);
 
 /* ------------------------------------------------------------------------
+ * Load balancing, training side.  Technical Report, Method: the router is
+ * balanced by the DeepSeek auxiliary-loss-free per-expert bias, stepped after
+ * each batch from the experts' loads, plus a sequence-wise balance loss
+ * against extreme imbalance inside one sequence.  The report names both and
+ * gives no formula; the published DeepSeek forms are taken (stated below).
+ *
+ * moe_balance_workspace_size -- bytes of workspace moe_balance_stats needs for
+ * dims->T tokens in sequences of seq_len tokens (0 on invalid arguments).
+ *
+ * moe_balance_stats -- per-sequence load statistics and the balance loss.
+ *   seq_len   tokens per sequence; T must be a whole number of sequences
+ *   probs     [T, E] fp32 softmax probabilities (moe_route / moe_forward)
+ *   topk_idx  [T, k] int32 chosen experts
+ *   alpha     balance-loss coefficient
+ *   f, P      [T/seq_len, E] fp32 out, for sequence s and expert e:
+ *               f[s,e] = E / (k seq_len) * #pairs of s routed to e
+ *               P[s,e] = mean over the tokens t of s of probs[t,e]
+ *   loss      [1] fp32 out: alpha * mean over s of sum_e f[s,e] P[s,e]
+ *             (0 when T == 0)
+ *   workspace moe_balance_workspace_size() bytes, 256-byte aligned
+ * Sums run in fp64 in a fixed order (deterministic); f is one rounding of the
+ * exact quotient.  An id outside [0, E) is skipped and recorded as
+ * MOE_ERR_INVALID_ARG in the device status word.  Returns INVALID_ARG (null
+ * pointer, seq_len <= 0, T not a multiple of seq_len), WORKSPACE, CUDA.
+ *
+ * moe_bias_update -- one auxiliary-loss-free bias step from a batch's loads:
+ *   counts    [E] int32 pairs per expert (the counts moe_permute and
+ *             moe_forward write); dims->T is the number of tokens they cover.
+ *             With data-parallel replicas the caller sums counts and T over
+ *             the replicas first, so that every replica takes the same step.
+ *   bias_out[e] = bias_in[e] - gamma  if E*counts[e] > T*k  (above the mean)
+ *                 bias_in[e] + gamma  if E*counts[e] < T*k  (below the mean)
+ *                 bias_in[e]          otherwise (bit for bit)
+ *   bias_out may alias bias_in.  The comparison is exact integer arithmetic;
+ *   the step is one fp32 rounding.  Returns INVALID_ARG (null pointer), CUDA.
+ * ---------------------------------------------------------------------- */
+size_t moe_balance_workspace_size(const moe_dims* dims, int seq_len);
+int moe_balance_stats(const moe_dims* dims, int seq_len, const float* probs,
+                      const int32_t* topk_idx, float alpha, float* f, float* P,
+                      float* loss, void* workspace, size_t workspace_bytes,
+                      void* stream);
+int moe_bias_update(const moe_dims* dims, const int32_t* counts, float gamma,
+                    const float* bias_in, float* bias_out, void* stream);
+
+/* ------------------------------------------------------------------------
  * Device status and bounded waits.
  *
  * moe_get_last_device_status: synchronises `stream`, returns the first error

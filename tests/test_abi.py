@@ -91,6 +91,32 @@ def test_null_pointers_and_workspace_rejected_on_host(lib):
     assert rc == M.MOE_ERR_INVALID_ARG
 
 
+def test_balance_calls_rejected_on_host(lib):
+    dm = M.dims(T=64, d=256, E=16, k=4, I=128, n_shared=2, align=16)
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: every call below fails first
+    assert lib.moe_balance_workspace_size(ctypes.byref(dm), 48) == 0   # 64 tokens % 48
+    assert lib.moe_balance_workspace_size(ctypes.byref(dm), 0) == 0
+    n = lib.moe_balance_workspace_size(ctypes.byref(dm), 16)           # 4 sequences
+    assert n >= 4 * 16 * (8 + 4) + 4 * 8
+    rc = lib.moe_balance_stats(ctypes.byref(dm), 48, fake, fake, 1.0, fake, fake, fake, fake,
+                               1 << 20, None)
+    assert rc == M.MOE_ERR_INVALID_ARG
+    rc = lib.moe_balance_stats(ctypes.byref(dm), 16, fake, fake, 1.0, fake, fake, fake, fake,
+                               16, None)
+    assert rc == M.MOE_ERR_WORKSPACE
+    rc = lib.moe_balance_stats(ctypes.byref(dm), 16, None, fake, 1.0, fake, fake, fake, fake,
+                               1 << 20, None)
+    assert rc == M.MOE_ERR_INVALID_ARG
+    misaligned = ctypes.c_void_p((1 << 20) + 8)
+    rc = lib.moe_balance_stats(ctypes.byref(dm), 16, fake, fake, 1.0, fake, fake, fake,
+                               misaligned, 1 << 20, None)
+    assert rc == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_bias_update(ctypes.byref(dm), None, 0.1, fake, fake, None) == \
+        M.MOE_ERR_INVALID_ARG
+    assert lib.moe_bias_update(ctypes.byref(dm), fake, 0.1, fake, None, None) == \
+        M.MOE_ERR_INVALID_ARG
+
+
 def test_status_strings(lib):
     for s in (0, -1, -2, -3, -4, -5):
         assert M.status_string(s) != "unknown status"

@@ -61,3 +61,53 @@ def test_whole_job_value_counts_all_ranks():
     assert bench.whole_job_value(2, 128, 10, 5.0) == pytest.approx(512000.0)
     assert bench.whole_job_value(1, 128, 10, 5.0) == pytest.approx(256000.0)
     assert bench.max_over_ranks(3.5, 1, "cpu") == 3.5
+
+
+def _loads_worker(rank, world, port, out):
+    """Each rank routes its own tokens; the bias step of the replicas uses the
+    loads summed over the group (fine_grained_moe_fp32_b200.moe.global_loads)."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import numpy as np
+    import bench
+    from fine_grained_moe_fp32_b200 import moe as M
+    from fine_grained_moe_fp32_b200.workloads import make_inputs, small_config
+    from oracle import moe_oracle as O
+
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        T = 24 + 8 * rank                       # ranks may hold different batch sizes
+        cfg = small_config(T=T, d=128, E=8, k=2, I=64)
+        inp = make_inputs(cfg, seed=bench.shard_seed(0, rank))
+        wts = make_inputs(cfg, seed=0)          # same router weights on every rank
+        idx = O.route(inp["x"], wts["w_gate"], wts["bias"], cfg.k)["idx"]
+        counts = torch.as_tensor(np.bincount(idx.ravel(), minlength=cfg.E), dtype=torch.int32)
+        c_all, T_all = M.global_loads(counts, T, group=dist.group.WORLD)
+        sizes = [None] * world
+        dist.all_gather_object(sizes, idx.tolist())
+        whole = np.concatenate([np.asarray(s) for s in sizes])
+        out[rank] = {"T_all": T_all, "c_all": c_all.tolist(),
+                     "c_whole": np.bincount(whole.ravel(), minlength=cfg.E).tolist(),
+                     "T_whole": whole.shape[0],
+                     "step": O.bias_update(wts["bias"], c_all.numpy(), 1e-3, T_all, cfg.k).tolist(),
+                     "step_whole": O.bias_update(wts["bias"], np.bincount(whole.ravel(),
+                                                 minlength=cfg.E), 1e-3, whole.shape[0],
+                                                 cfg.k).tolist()}
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_bias_step_uses_global_loads_on_gloo():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.start_processes(_loads_worker, args=(world, port, out), nprocs=world, join=True,
+                           start_method="spawn")
+        res = dict(out)
+    assert set(res) == {0, 1}
+    for r in range(world):
+        assert res[r]["T_all"] == res[r]["T_whole"] == 24 + 32
+        assert res[r]["c_all"] == res[r]["c_whole"]
+        assert res[r]["step"] == res[r]["step_whole"]
+    assert res[0]["step"] == res[1]["step"]      # every replica takes the same step
