@@ -39,7 +39,7 @@ from fine_grained_moe_fp32_b200.workloads import CONFIGS, make_inputs  # noqa: E
 METRIC = "MoE-layer tokens/s (bf16, d=5120, 128E top-6 + 2 shared) and % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNELS_PER_STEP = 9  # router gemm + top-k, 4 permutation kernels, 2 grouped GEMMs, combine
-BWD_KERNELS = 12      # combine/router bwd (3), 5 grouped GEMMs, 2 gate GEMMs + split sum, un-permute
+BWD_KERNELS = 11      # combine/router bwd (3), 4 grouped GEMMs (dW1 and dW3 in one), 2 gate GEMMs + split sum, un-permute
 BALANCE_KERNELS = 4   # balance partial sums, per-sequence f/P, loss, bias step
 # training-side balancing of the fwd+bwd step: sequences of the 8K pretraining
 # context (Technical Report, Results: 8K extended to 32K later); the loss

@@ -57,6 +57,11 @@ struct BwdParams {
   int kit_routed, kit_shared;          // dgrad: K chunks of 64
   int ksplit_routed, ksplit_shared;    // dgrad-up: first chunk read from the second A map
   int a_col0_routed, a_col0_shared, a_step_shared;  // wgrad: A column offsets
+  // wgrad: M tiles at or past m_split belong to a second output (out2_*),
+  // their A columns start at a_col1_* (0 = one output)
+  int m_split;
+  int a_col1_routed, a_col1_shared;
+  void *out2_routed, *out2_shared;
   int b_col0_routed, b_col0_shared, b_step_shared;  // wgrad: B column offsets
   void* out_routed;
   int ld_routed;
@@ -306,12 +311,16 @@ grouped_gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmA_r,
             // wgrad: A (M columns) and B (N columns) of token-major sources, K = tokens
             const int nblk = t.n / 64;
             mbar_arrive_expect_tx(fb, kABytes + nblk * 8192);
-            const int acol = routed ? p.a_col0_routed : p.a_col0_shared + s_idx * p.a_step_shared;
+            const bool second = p.m_split > 0 && t.mt >= p.m_split;
+            const int mt = second ? t.mt - p.m_split : t.mt;
+            const int acol = second
+                ? (routed ? p.a_col1_routed : p.a_col1_shared + s_idx * p.a_step_shared)
+                : (routed ? p.a_col0_routed : p.a_col0_shared + s_idx * p.a_step_shared);
             const int bcol = routed ? p.b_col0_routed : p.b_col0_shared + s_idx * p.b_step_shared;
             const CUtensorMap* tA = routed ? &tmA_r : &tmA_s;
             const CUtensorMap* tB = routed ? &tmB_r : &tmB_s;
             for (int h = 0; h < 2; ++h)
-              tma_load_3d(sA + h * 8192, tA, fb, acol + t.mt * 128 + h * 64, t.row0 + kk, 0, pol_b);
+              tma_load_3d(sA + h * 8192, tA, fb, acol + mt * 128 + h * 64, t.row0 + kk, 0, pol_b);
             for (int j = 0; j < nblk; ++j)
               tma_load_3d(sB + j * 8192, tB, fb, bcol + t.ncol0 + j * 64, t.row0 + kk, 0, pol_b);
           }
@@ -377,8 +386,33 @@ grouped_gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmA_r,
     const int mrow = q * 32 + lane;  // accumulator row = TMEM lane
     int acc = 0;
     uint32_t acc_phase = 0;
+    const int et = threadIdx.x - 64;  // 0..127 over the epilogue warps
+    // SwiGLU backward: this thread's share of the g / u rows of one 32-token
+    // chunk (4 x 16 bytes each), loaded a chunk ahead so the global latency
+    // overlaps the accumulator wait and the previous chunk's work
+    uint4 gpre[4], upre[4];
+    auto load_gu = [&](const Tile& t, int c0) {
+      const bool routed = t.g < p.E;
+      const uint16_t* gsrc = routed ? p.g_routed : p.g_shared;
+      const uint16_t* usrc = routed ? p.u_routed : p.u_shared;
+      const int ldgu = routed ? p.ld_gu_routed : p.ld_gu_shared;
+      const int nj = min(32, t.nrows - c0);
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {
+        const int i = et + it * kEpiThreads;
+        const int r = i >> 4, cv = i & 15;
+        gpre[it] = make_uint4(0, 0, 0, 0);
+        upre[it] = gpre[it];
+        if (r < nj) {
+          const size_t at = (size_t)(t.row0 + c0 + r) * ldgu + t.mt * 128 + cv * 8;
+          gpre[it] = *reinterpret_cast<const uint4*>(gsrc + at);
+          upre[it] = *reinterpret_cast<const uint4*>(usrc + at);
+        }
+      }
+    };
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       const Tile t = decode<MODE>(ctl, p, tile);
+      if (MODE == kDgradDown) load_gu(t, 0);
       bool bad = aborted(ctl);
       if (!bad && !mbar_wait_bounded(smem_u32(&ctl.tfull[acc]), acc_phase, p.wait_limit_ns)) {
         record_timeout(ctl, p);
@@ -396,11 +430,15 @@ grouped_gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmA_r,
         const int nj = min(32, ncols - c0);
         if (MODE == kWgrad) {
           // dW[group][mt*128 + mrow][ncol0 + c0 + j], bf16, 16-byte stores
-          uint16_t* out = static_cast<uint16_t*>(routed ? p.out_routed : p.out_shared);
+          const bool second = p.m_split > 0 && t.mt >= p.m_split;
+          const int mt = second ? t.mt - p.m_split : t.mt;
+          uint16_t* out = static_cast<uint16_t*>(
+              second ? (routed ? p.out2_routed : p.out2_shared)
+                     : (routed ? p.out_routed : p.out_shared));
           const int ldo = routed ? p.ntot_routed : p.ntot_shared;
           const int64_t gbase = routed ? (int64_t)t.g * p.gstride_routed
                                        : (int64_t)(t.g - p.E) * p.gstride_shared;
-          uint16_t* dst = out + gbase + (int64_t)(t.mt * 128 + mrow) * ldo + t.ncol0 + c0;
+          uint16_t* dst = out + gbase + (int64_t)(mt * 128 + mrow) * ldo + t.ncol0 + c0;
           const bool zero = t.kchunks == 0;  // no tokens: the gradient is zero
 #pragma unroll
           for (int j8 = 0; j8 < 4; ++j8) {
@@ -421,25 +459,18 @@ grouped_gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmA_r,
           // g and u come in, and dG / dU go out, as coalesced 16-byte rows;
           // each thread then works on its own feature (TMEM lane) in place.
           const int f0 = t.mt * 128;
-          const uint16_t* gsrc = routed ? p.g_routed : p.g_shared;
-          const uint16_t* usrc = routed ? p.u_routed : p.u_shared;
-          const int ldgu = routed ? p.ld_gu_routed : p.ld_gu_shared;
           uint16_t* out = static_cast<uint16_t*>(routed ? p.out_routed : p.out_shared);
           const int ldo = routed ? p.ld_routed : p.ld_shared;
           const int ucol = routed ? p.ucol_routed : p.ucol_shared;
-          const int et = threadIdx.x - 64;  // 0..127 over the epilogue warps
-          for (int i = et; i < 32 * 16; i += kEpiThreads) {
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            const int i = et + it * kEpiThreads;
             const int r = i >> 4, cv = i & 15;
-            uint4 gv = make_uint4(0, 0, 0, 0), uv = gv;
-            if (r < nj) {
-              const size_t at = (size_t)(t.row0 + c0 + r) * ldgu + f0 + cv * 8;
-              gv = *reinterpret_cast<const uint4*>(gsrc + at);
-              uv = *reinterpret_cast<const uint4*>(usrc + at);
-            }
-            *reinterpret_cast<uint4*>(epi_g + r * 128 + cv * 8) = gv;
-            *reinterpret_cast<uint4*>(epi_u + r * 128 + cv * 8) = uv;
+            *reinterpret_cast<uint4*>(epi_g + r * 128 + cv * 8) = gpre[it];
+            *reinterpret_cast<uint4*>(epi_u + r * 128 + cv * 8) = upre[it];
           }
           named_bar_sync(1, kEpiThreads);
+          if (c0 + 32 < ncols) load_gu(t, c0 + 32);  // next chunk, in flight meanwhile
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (j < nj) {
@@ -655,8 +686,10 @@ cudaError_t launch_backward_gemms(const Shape& s, const BackwardGemmArgs& a, int
     if ((err = launch_bwd<kDgradUp>(m, p, num_sms, st)) != cudaSuccess) return err;
     if ((err = mark(2)) != cudaSuccess) return err;
   }
-  // ---- dW1 = dG^T X, dW3 = dU^T X (routed: x_perm; shared: x)
-  for (int which = 0; which < 2; ++which) {
+  // ---- dW1 = dG^T X and dW3 = dU^T X in one launch (routed: x_perm;
+  // shared: x): M tiles [0, I/128) write dW1, [I/128, 2I/128) write dW3, and
+  // both halves stream the same token panels
+  {
     bool ok = make_map3(&m[0], a.dgu_perm, 2 * (uint64_t)s.I, s.cap, 1, 64) &&
               make_map3(&m[2], a.x_perm, s.d, s.cap, 1, 64);
     m[1] = m[0];
@@ -669,17 +702,22 @@ cudaError_t launch_backward_gemms(const Shape& s, const BackwardGemmArgs& a, int
     if (!ok) return cudaErrorInvalidValue;
     BwdParams p = base_params(s, a.offsets, status, wait_ns);
     p.n_sgroups = shared ? s.S : 0;
-    p.mt_routed = p.mt_shared = s.I / 128;
+    p.mt_routed = p.mt_shared = 2 * s.I / 128;
+    p.m_split = s.I / 128;
     p.ntot_routed = p.ntot_shared = s.d;
     p.nt_routed = p.nt_shared = (int)ceil_div(s.d, kNT);
-    p.a_col0_routed = which == 0 ? 0 : s.I;
-    p.a_col0_shared = which == 0 ? 0 : SI;
+    p.a_col0_routed = 0;
+    p.a_col1_routed = s.I;
+    p.a_col0_shared = 0;
+    p.a_col1_shared = SI;
     p.a_step_shared = s.I;
     p.b_col0_routed = 0;
     p.b_col0_shared = 0;
     p.b_step_shared = 0;
-    p.out_routed = which == 0 ? a.dw1 : a.dw3;
-    p.out_shared = which == 0 ? a.dws1 : a.dws3;
+    p.out_routed = a.dw1;
+    p.out2_routed = a.dw3;
+    p.out_shared = a.dws1;
+    p.out2_shared = a.dws3;
     p.gstride_routed = p.gstride_shared = (int64_t)s.I * s.d;
     if ((err = launch_bwd<kWgrad>(m, p, num_sms, st)) != cudaSuccess) return err;
   }
