@@ -582,6 +582,10 @@ BwdParams base_params(const Shape& s, const int32_t* offsets, unsigned int* stat
 cudaError_t launch_backward_gemms(const Shape& s, const BackwardGemmArgs& a, int num_sms,
                                   unsigned int* status, uint64_t wait_ns, cudaStream_t st,
                                   const cudaEvent_t* events) {
+  // prefill-sized segments run on CTA pairs (grouped_gemm_bwd_pair.cu)
+  const bool small = (int64_t)s.T * s.k <= (int64_t)24 * s.E;
+  if (!small && pair_backward_supported(s))
+    return launch_backward_gemms_pair(s, a, num_sms, status, wait_ns, st, events);
   auto mark = [&](int i) {
     return events != nullptr ? cudaEventRecord(events[i], st) : cudaSuccess;
   };

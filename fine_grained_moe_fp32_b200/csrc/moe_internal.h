@@ -86,6 +86,10 @@ struct BackwardGemmArgs {
 };
 // `events` (may be null): 4 events recorded after the dH/SwiGLU dgrad, the dW2
 // wgrad, the dX dgrad and the dW1/dW3 wgrads.
+bool pair_backward_supported(const Shape& s);
+cudaError_t launch_backward_gemms_pair(const Shape& s, const BackwardGemmArgs& a, int num_sms,
+                                       unsigned int* status, uint64_t wait_ns, cudaStream_t st,
+                                       const cudaEvent_t* events);
 cudaError_t launch_backward_gemms(const Shape& s, const BackwardGemmArgs& a, int num_sms,
                                   unsigned int* status, uint64_t wait_ns, cudaStream_t st,
                                   const cudaEvent_t* events = nullptr);

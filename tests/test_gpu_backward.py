@@ -89,6 +89,8 @@ CASES = [
     ("small_E16_T200", small_config(T=200, d=256, E=16, k=4, I=128), None),
     ("E32_S1_k8_T97", MoEConfig("s1k8", T=97, d=384, E=32, k=8, S=1, I=256, bias="normal0.05"),
      None),
+    # ~256 rows per expert: several token tiles per dgrad, several K chunks per wgrad
+    ("E8_k2_T1024_long_segments", small_config(T=1024, d=256, E=8, k=2, I=128), None),
 ]
 
 
@@ -105,12 +107,15 @@ def test_backward_parity_small(name, cfg, T):
         assert not grads["dw1"][e].any() and not grads["dw2"][e].any()
 
 
-def test_backward_full_size_slice():
+@pytest.mark.parametrize("T", [256, 1024], ids=["T256_one_cta", "T1024_cta_pairs"])
+def test_backward_full_size_slice(T):
     """The fwd+bwd workload's layer (d=5120, E=128, I=1408, 2 shared) on its
-    first 256 tokens: dx, dWg and the shared experts' gradients in full, the
-    routed experts' gradients on a seeded sample of experts."""
+    first T tokens (256: the one-CTA GEMMs for decode-sized segments; 1024:
+    the paired-CTA GEMMs of prefill-sized batches): dx, dWg and the shared
+    experts' gradients in full, the routed experts' gradients on a seeded
+    sample of experts."""
     cfg = CONFIGS[4]
-    inp = make_inputs(cfg, T=256, device="cuda")
+    inp = make_inputs(cfg, T=T, device="cuda")
     y_inf, y, grads, idx = _run(inp)
     rng = np.random.default_rng(4)
     experts = sorted(set(rng.choice(cfg.E, size=6, replace=False).tolist()) | {int(idx[0, 0])})
