@@ -186,8 +186,8 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
   const uint32_t raw = smem_u32(dsmem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   // epilogue staging, 16 KB: the SwiGLU backward's g then u tiles ([32][128]
-  // bf16 each), or the weight gradients' two 8 KB store buffers (128 rows x
-  // 32 columns of bf16, 64-byte swizzle)
+  // bf16 each), or per epilogue warp two 2 KB store buffers of the weight
+  // gradients (32 rows x 32 columns of bf16, 64-byte swizzle)
   uint8_t* epi = dsmem_raw + (sbase - raw) + kStages * kStageBytes;
   uint16_t* epi_g = reinterpret_cast<uint16_t*>(epi);
   uint16_t* epi_u = epi_g + 32 * 128;
@@ -486,20 +486,19 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
       tc_fence_after();
       const uint32_t tbase = tmem_base + (uint32_t)(acc * kNT) + ((uint32_t)(q * 32) << 16);
       const int ncols = MODE == kPWgrad ? t.n : t.nrows;
-      for (int c0 = 0; live && c0 < ncols; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tbase + (uint32_t)c0, v);
-        tmem_ld_wait();
-        const int nj = min(32, ncols - c0);
-        if (MODE == kPWgrad) {
-          // dW[group][row0 + mrow][ncol0 + c0 .. + 32] in bf16: each thread
-          // writes its row's 64 bytes into a staging buffer, one thread hands
-          // the 128 x 32 block to a TMA store (whole rows, coalesced); two
-          // buffers alternate so the store of one overlaps the next chunk
-          const bool second = p.a_split > 0 && r0 >= p.a_split;
-          const CUtensorMap* tO =
-              second ? (routed ? &tmO2_r : &tmO2_s) : (routed ? &tmO_r : &tmO_s);
-          const bool zero = t.kchunks == 0;  // no tokens: the gradient is zero
+      if (MODE == kPWgrad && live) {
+        // dW[group][row0 + mrow][ncol0 + c0 .. + 32] in bf16.  Each warp owns
+        // 32 rows: it stages its 32 x 32 block (64-byte rows, 64-byte
+        // swizzle) and hands it to a TMA store (whole rows, coalesced) with
+        // warp-level syncs only; its two buffers alternate, and the TMEM load
+        // of the next chunk is in flight while this one is packed and staged.
+        const bool second = p.a_split > 0 && r0 >= p.a_split;
+        const CUtensorMap* tO =
+            second ? (routed ? &tmO2_r : &tmO2_s) : (routed ? &tmO_r : &tmO_s);
+        const int orow = (second ? r0 - p.a_split : r0) + q * 32;
+        const int plane = routed ? t.g : t.g - p.E;
+        const bool zero = t.kchunks == 0;  // no tokens: the gradient is zero
+        auto stage_store = [&](const uint32_t (&v)[32], int c0) {
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -508,24 +507,43 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
             w[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
                    ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
           }
-          uint8_t* buf = epi + (nstore & 1u) * 8192u;
-          if (et == 0) bulk_wait_group_read<1>();  // the store that last used buf has read it
-          named_bar_sync(1, kEpiThreads);
+          uint8_t* buf = epi + q * 4096 + (nstore & 1u) * 2048u;
+          if (lane == 0) bulk_wait_group_read<1>();  // the store that last used buf has read it
+          __syncwarp();
 #pragma unroll
           for (int c = 0; c < 4; ++c) {  // 64-byte swizzle: 16-byte chunk c ^ ((row / 2) % 4)
-            const int phys = c ^ ((mrow >> 1) & 3);
-            *reinterpret_cast<uint4*>(buf + mrow * 64 + phys * 16) =
+            const int phys = c ^ ((lane >> 1) & 3);
+            *reinterpret_cast<uint4*>(buf + lane * 64 + phys * 16) =
                 make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
           }
           fence_proxy_async_smem();
-          named_bar_sync(1, kEpiThreads);
-          if (et == 0) {
-            tma_store_3d(tO, smem_u32(buf), t.ncol0 + c0, second ? r0 - p.a_split : r0,
-                         routed ? t.g : t.g - p.E);
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(tO, smem_u32(buf), t.ncol0 + c0, orow, plane);
             bulk_commit_group();
           }
           ++nstore;
-        } else if (MODE == kPDgradDown) {
+        };
+        // tile widths are multiples of 64: chunks go in pairs (va, vb)
+        uint32_t va[32], vb[32];
+        tmem_ld_32x32b_x32(tbase, va);
+        tmem_ld_wait();
+        for (int c0 = 0; c0 < ncols; c0 += 64) {
+          tmem_ld_32x32b_x32(tbase + (uint32_t)(c0 + 32), vb);
+          stage_store(va, c0);
+          tmem_ld_wait();
+          const bool more = c0 + 64 < ncols;
+          if (more) tmem_ld_32x32b_x32(tbase + (uint32_t)(c0 + 64), va);
+          stage_store(vb, c0 + 32);
+          if (more) tmem_ld_wait();
+        }
+      }
+      for (int c0 = 0; MODE != kPWgrad && live && c0 < ncols; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tbase + (uint32_t)c0, v);
+        tmem_ld_wait();
+        const int nj = min(32, ncols - c0);
+        if (MODE == kPDgradDown) {
           // SwiGLU backward on a 32-token x 128-feature tile staged in smem
           uint16_t* out = static_cast<uint16_t*>(routed ? p.out_routed : p.out_shared);
           const int ldo = routed ? p.ld_routed : p.ld_shared;
@@ -581,7 +599,7 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
         mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
-    if (MODE == kPWgrad && et == 0) bulk_wait_group<0>();  // every store has landed
+    if (MODE == kPWgrad && lane == 0) bulk_wait_group<0>();  // every store has landed
   }
 
   tc_fence_before();
@@ -623,14 +641,14 @@ bool make_map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 output (inner, rows, planes) written by TMA stores of 32 x 128 boxes,
+// bf16 output (inner, rows, planes) written by TMA stores of 32 x 32 boxes,
 // 64-byte swizzle (the staging layout of the weight-gradient epilogue).
 bool make_store_map3(CUtensorMap* m, void* base, uint64_t inner, uint64_t rows, uint64_t planes) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {inner, rows, planes};
   cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
-  cuuint32_t box[3] = {32u, 128u, 1u};
+  cuuint32_t box[3] = {32u, 32u, 1u};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
