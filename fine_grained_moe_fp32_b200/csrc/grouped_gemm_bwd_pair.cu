@@ -185,9 +185,9 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
   extern __shared__ uint8_t dsmem_raw[];
   const uint32_t raw = smem_u32(dsmem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
-  // epilogue staging, 16 KB: the SwiGLU backward's g then u tiles ([32][128]
-  // bf16 each), or per epilogue warp two 2 KB store buffers of the weight
-  // gradients (32 rows x 32 columns of bf16, 64-byte swizzle)
+  // epilogue staging, 32 KB: the SwiGLU backward's g then u tiles ([32][128]
+  // bf16 each), or per epilogue warp two 4 KB store buffers of the weight
+  // gradients (32 rows x 64 columns of bf16, 128-byte swizzle)
   uint8_t* epi = dsmem_raw + (sbase - raw) + kStages * kStageBytes;
   uint16_t* epi_g = reinterpret_cast<uint16_t*>(epi);
   uint16_t* epi_u = epi_g + 32 * 128;
@@ -487,19 +487,18 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
       const uint32_t tbase = tmem_base + (uint32_t)(acc * kNT) + ((uint32_t)(q * 32) << 16);
       const int ncols = MODE == kPWgrad ? t.n : t.nrows;
       if (MODE == kPWgrad && live) {
-        // dW[group][row0 + mrow][ncol0 + c0 .. + 32] in bf16.  Each warp owns
-        // 32 rows: it stages its 32 x 32 block (64-byte rows, 64-byte
+        // dW[group][row0 + mrow][ncol0 + c0 .. + 64] in bf16.  Each warp owns
+        // 32 rows: it stages its 32 x 64 block (128-byte rows, 128-byte
         // swizzle) and hands it to a TMA store (whole rows, coalesced) with
-        // warp-level syncs only; its two buffers alternate, and the TMEM load
-        // of the next chunk is in flight while this one is packed and staged.
+        // warp-level syncs only; its two buffers alternate, and the TMEM loads
+        // of the next 64 columns are in flight while these are staged.
         const bool second = p.a_split > 0 && r0 >= p.a_split;
         const CUtensorMap* tO =
             second ? (routed ? &tmO2_r : &tmO2_s) : (routed ? &tmO_r : &tmO_s);
         const int orow = (second ? r0 - p.a_split : r0) + q * 32;
         const int plane = routed ? t.g : t.g - p.E;
         const bool zero = t.kchunks == 0;  // no tokens: the gradient is zero
-        auto stage_store = [&](const uint32_t (&v)[32], int c0) {
-          uint32_t w[16];
+        auto pack = [&](const uint32_t (&v)[32], uint32_t (&w)[16]) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float lo = zero ? 0.f : __uint_as_float(v[2 * i]);
@@ -507,14 +506,30 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
             w[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
                    ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
           }
-          uint8_t* buf = epi + q * 4096 + (nstore & 1u) * 2048u;
+        };
+        // tile widths are multiples of 64: columns go 64 at a time (va, vb)
+        uint32_t va[32], vb[32];
+        tmem_ld_32x32b_x32(tbase, va);
+        tmem_ld_32x32b_x32(tbase + 32u, vb);
+        tmem_ld_wait();
+        for (int c0 = 0; c0 < ncols; c0 += 64) {
+          uint32_t wa[16], wb[16];
+          pack(va, wa);
+          pack(vb, wb);
+          const bool more = c0 + 64 < ncols;
+          if (more) {
+            tmem_ld_32x32b_x32(tbase + (uint32_t)(c0 + 64), va);
+            tmem_ld_32x32b_x32(tbase + (uint32_t)(c0 + 96), vb);
+          }
+          uint8_t* buf = epi + q * 8192 + (nstore & 1u) * 4096u;
           if (lane == 0) bulk_wait_group_read<1>();  // the store that last used buf has read it
           __syncwarp();
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {  // 64-byte swizzle: 16-byte chunk c ^ ((row / 2) % 4)
-            const int phys = c ^ ((lane >> 1) & 3);
-            *reinterpret_cast<uint4*>(buf + lane * 64 + phys * 16) =
-                make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+          for (int c = 0; c < 8; ++c) {  // 128-byte swizzle: 16-byte chunk c ^ (row % 8)
+            const int phys = c ^ (lane & 7);
+            const uint32_t* w = c < 4 ? &wa[4 * c] : &wb[4 * (c - 4)];
+            *reinterpret_cast<uint4*>(buf + lane * 128 + phys * 16) =
+                make_uint4(w[0], w[1], w[2], w[3]);
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -523,18 +538,6 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
             bulk_commit_group();
           }
           ++nstore;
-        };
-        // tile widths are multiples of 64: chunks go in pairs (va, vb)
-        uint32_t va[32], vb[32];
-        tmem_ld_32x32b_x32(tbase, va);
-        tmem_ld_wait();
-        for (int c0 = 0; c0 < ncols; c0 += 64) {
-          tmem_ld_32x32b_x32(tbase + (uint32_t)(c0 + 32), vb);
-          stage_store(va, c0);
-          tmem_ld_wait();
-          const bool more = c0 + 64 < ncols;
-          if (more) tmem_ld_32x32b_x32(tbase + (uint32_t)(c0 + 64), va);
-          stage_store(vb, c0 + 32);
           if (more) tmem_ld_wait();
         }
       }
@@ -641,24 +644,24 @@ bool make_map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 output (inner, rows, planes) written by TMA stores of 32 x 32 boxes,
-// 64-byte swizzle (the staging layout of the weight-gradient epilogue).
+// bf16 output (inner, rows, planes) written by TMA stores of 64 x 32 boxes,
+// 128-byte swizzle (the staging layout of the weight-gradient epilogue).
 bool make_store_map3(CUtensorMap* m, void* base, uint64_t inner, uint64_t rows, uint64_t planes) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {inner, rows, planes};
   cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
-  cuuint32_t box[3] = {32u, 32u, 1u};
+  cuuint32_t box[3] = {64u, 32u, 1u};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // m[0..5]: operand maps; m[6..9]: output maps of the weight gradients.
 template <int MODE>
 cudaError_t launch_pb(const CUtensorMap* m, const PBParams& p, int num_sms, cudaStream_t st) {
-  constexpr size_t smem = (size_t)kStages * kStageBytes + 2 * 32 * 128 * 2 + 1024;
+  constexpr size_t smem = (size_t)kStages * kStageBytes + 32768 + 1024;
   static_assert(smem + sizeof(PBCtl) <= 232448, "shared memory budget");
   auto kern = grouped_gemm_bwd_pair_kernel<MODE>;
   cudaError_t err =
