@@ -38,7 +38,11 @@ from fine_grained_moe_fp32_b200.workloads import CONFIGS, make_inputs  # noqa: E
 
 METRIC = "MoE-layer tokens/s (bf16, d=5120, 128E top-6 + 2 shared) and % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 9  # router gemm + top-k, 4 permutation kernels, 2 grouped GEMMs, combine
+def forward_kernels(T: int) -> int:
+    """Launches of one moe_forward: router GEMM + top-k, the permutation (one
+    index kernel + gather for a batch of at most 256 tokens, else count, scan,
+    scatter + gather), the two grouped GEMMs, the combine."""
+    return 2 + (2 if T <= 256 else 4) + 2 + 1
 BWD_KERNELS = 11      # combine/router bwd (3), 4 grouped GEMMs (dW1 and dW3 in one), 2 gate GEMMs + split sum, un-permute
 BALANCE_KERNELS = 4   # balance partial sums, per-sequence f/P, loss, bias step
 # training-side balancing of the fwd+bwd step: sequences of the 8K pretraining
@@ -461,7 +465,7 @@ def run_ours(args):
         "e2e": {"value": e2e_value, "unit": "tokens/s",
                 "h2d_bytes_per_step": T * cfg.d * 2 * (2 if train else 1),
                 "d2h_bytes_per_step": T * cfg.d * 2},
-        "gpu_launches": (KERNELS_PER_STEP + (BWD_KERNELS + BALANCE_KERNELS if train else 0))
+        "gpu_launches": (forward_kernels(T) + (BWD_KERNELS + BALANCE_KERNELS if train else 0))
         * args.steps,
     }
     if train:

@@ -4,8 +4,9 @@
 //
 //   y[t] = y_shared[t] + sum_{j < k} w[t, j] * y_perm[row_of[t*k + j]]
 //
-// fp32 accumulation, slot j in ascending order, one rounding to bf16.  One CTA
-// per token; 16-byte vectors (8 bf16) along the hidden dimension.
+// fp32 accumulation, slot j in ascending order, one rounding to bf16.  CTA
+// (t, b) covers 16-byte vectors (8 bf16) b*128 .. b*128+127 of token t, one
+// per thread, with the k routed rows' loads all issued before the sum.
 #include <cuda_bf16.h>
 
 #include "moe_internal.h"
@@ -39,7 +40,8 @@ combine_kernel(const uint16_t* __restrict__ y_perm, const int32_t* __restrict__ 
   }
   __syncthreads();
   const int nv = d / 8;
-  for (int v = threadIdx.x; v < nv; v += kThreads) {
+  const int v = blockIdx.y * kThreads + threadIdx.x;
+  if (v < nv) {
     float acc[8];
     if (y_shared != nullptr) {
       const float4* s = reinterpret_cast<const float4*>(y_shared + (size_t)t * d) + 2 * v;
@@ -50,11 +52,14 @@ combine_kernel(const uint16_t* __restrict__ y_perm, const int32_t* __restrict__ 
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
     }
-    for (int j = 0; j < k; ++j) {
-      if (rows[j] < 0) continue;
-      const uint4 val = reinterpret_cast<const uint4*>(y_perm + (size_t)rows[j] * d)[v];
-      add_bf16x8(acc, val, ws[j]);
-    }
+    uint4 val[kMaxK];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (j < k && rows[j] >= 0)
+        val[j] = reinterpret_cast<const uint4*>(y_perm + (size_t)rows[j] * d)[v];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (j < k && rows[j] >= 0) add_bf16x8(acc, val[j], ws[j]);
     uint32_t o[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -72,7 +77,8 @@ cudaError_t launch_combine(const Shape& s, const uint16_t* y_perm, const int32_t
                            const float* topk_w, const float* y_shared, uint16_t* y,
                            cudaStream_t st) {
   if (s.T == 0) return cudaSuccess;
-  combine_kernel<<<s.T, kThreads, 0, st>>>(y_perm, row_of, topk_w, y_shared, y, s.d, s.k, s.cap);
+  const dim3 grid((unsigned)s.T, (unsigned)ceil_div(s.d / 8, kThreads));
+  combine_kernel<<<grid, kThreads, 0, st>>>(y_perm, row_of, topk_w, y_shared, y, s.d, s.k, s.cap);
   return cudaGetLastError();
 }
 

@@ -10,6 +10,10 @@
 //                           masks + per-warp prefix), row_of / token_of_row
 //   permute_gather_kernel   one warp per row: x_perm[r] = x[token_of_row[r]]
 //                           (zero for padding rows), 16-byte vectors
+//
+// A batch of at most one chunk (decode) runs count, scan and scatter as one
+// CTA (permute_index_one_chunk_kernel): the same ranks and rows, two launches
+// fewer.
 #include "moe_internal.h"
 
 namespace moe {
@@ -129,6 +133,83 @@ permute_scatter_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
   }
 }
 
+// count + scan + scatter for T <= kChunk tokens in one CTA of kChunk threads
+// (token t = thread t): the per-warp ballot masks give both each expert's
+// count and each pair's rank among earlier tokens.
+__global__ void __launch_bounds__(kChunk)
+permute_index_one_chunk_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int align,
+                               int64_t cap, int32_t* __restrict__ counts,
+                               int32_t* __restrict__ offsets, int32_t* __restrict__ row_of,
+                               int32_t* __restrict__ token_of_row, unsigned int* status) {
+  __shared__ unsigned int masks[kWarps][kMaxE];
+  __shared__ int pre[kWarps][kMaxE];
+  __shared__ int scan[kMaxE];
+  __shared__ int base[kMaxE];
+  const int t = threadIdx.x;
+  const int warp = t >> 5, lane = t & 31;
+  for (int i = t; i < kWarps * kMaxE; i += blockDim.x) (&masks[0][0])[i] = 0u;
+  __syncthreads();
+  const bool tok_ok = t < T;
+  if (tok_ok) {
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      bool dup = false;
+      for (int jj = 0; jj < j; ++jj) dup |= idx[(size_t)t * k + jj] == e;
+      if (e >= 0 && e < E && !dup)
+        atomicOr(&masks[warp][e], 1u << lane);
+      else
+        set_status(status, DEV_BAD_EXPERT_ID);
+    }
+  }
+  __syncthreads();
+  int total = 0, padded = 0;
+  if (t < kMaxE) {
+    if (t < E) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        pre[w][t] = total;
+        total += __popc(masks[w][t]);
+      }
+      counts[t] = total;
+      padded = (int)round_up(total, align);
+    }
+    scan[t] = padded;
+  }
+  __syncthreads();
+  // inclusive Hillis-Steele scan over the (at most 128) experts
+  for (int o = 1; o < kMaxE; o <<= 1) {
+    const int v = (t < kMaxE && t >= o) ? scan[t - o] : 0;
+    __syncthreads();
+    if (t < kMaxE) scan[t] += v;
+    __syncthreads();
+  }
+  if (t < E) {
+    const int end = scan[t];
+    const int start = end - padded;
+    offsets[t] = start;
+    if (t == E - 1) offsets[E] = end;
+    base[t] = start;
+    for (int r = start + total; r < end; ++r) token_of_row[r] = -1;
+  }
+  const int used = scan[E - 1];
+  for (int64_t r = used + t; r < cap; r += blockDim.x) token_of_row[r] = -1;
+  __syncthreads();
+  if (tok_ok) {
+    const unsigned int lt = (1u << lane) - 1u;
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      bool dup = false;
+      for (int jj = 0; jj < j; ++jj) dup |= idx[(size_t)t * k + jj] == e;
+      int row = -1;
+      if (e >= 0 && e < E && !dup) {
+        row = base[e] + pre[warp][e] + __popc(masks[warp][e] & lt);
+        token_of_row[row] = t;
+      }
+      row_of[(size_t)t * k + j] = row;
+    }
+  }
+}
+
 constexpr int kGatherWarps = 8;
 
 __global__ void __launch_bounds__(kGatherWarps * 32)
@@ -165,15 +246,21 @@ cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16
   const int nchunks = (int)ceil_div(s.T, kChunk);
   int32_t* chunk_counts = static_cast<int32_t*>(scratch);
   int32_t* chunk_base = chunk_counts + (size_t)nchunks * s.E;
-  if (nchunks > 0) {
-    permute_count_kernel<<<nchunks, kChunk, 0, st>>>(topk_idx, s.T, s.k, s.E, chunk_counts,
-                                                     status);
-  }
-  permute_scan_kernel<<<1, kMaxE, 0, st>>>(chunk_counts, nchunks, s.E, s.align, s.cap,
-                                           chunk_base, counts, offsets, token_of_row);
-  if (nchunks > 0) {
-    permute_scatter_kernel<<<nchunks, kChunk, 0, st>>>(topk_idx, s.T, s.k, s.E, chunk_base,
-                                                       offsets, row_of, token_of_row);
+  if (nchunks == 1) {
+    permute_index_one_chunk_kernel<<<1, kChunk, 0, st>>>(topk_idx, s.T, s.k, s.E, s.align, s.cap,
+                                                         counts, offsets, row_of, token_of_row,
+                                                         status);
+  } else {
+    if (nchunks > 0) {
+      permute_count_kernel<<<nchunks, kChunk, 0, st>>>(topk_idx, s.T, s.k, s.E, chunk_counts,
+                                                       status);
+    }
+    permute_scan_kernel<<<1, kMaxE, 0, st>>>(chunk_counts, nchunks, s.E, s.align, s.cap,
+                                             chunk_base, counts, offsets, token_of_row);
+    if (nchunks > 0) {
+      permute_scatter_kernel<<<nchunks, kChunk, 0, st>>>(topk_idx, s.T, s.k, s.E, chunk_base,
+                                                         offsets, row_of, token_of_row);
+    }
   }
   if (s.cap > 0 && x_perm != nullptr) {
     const unsigned blocks = (unsigned)ceil_div(s.cap, kGatherWarps);

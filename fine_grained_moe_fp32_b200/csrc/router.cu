@@ -149,6 +149,101 @@ router_gemm_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wg,
   }
 }
 
+// Decode-sized batches (one token tile, K slices of 64): the CTA's whole
+// slice of x and w_gate is loaded at once -- one memory round trip instead of
+// four -- and each output is summed in fp32 from zero over its 64 products in
+// ascending k, the same group the streaming kernel forms, so the partials are
+// bit-identical to that kernel's.
+constexpr int kOneShotK = 64;
+constexpr size_t kOneShotSmem = (size_t)kOneShotK * (BT + BE) * sizeof(float);
+
+__global__ void __launch_bounds__(kThreads, 1)
+router_gemm_oneshot_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wg,
+                           float* __restrict__ part, int T, int d, int E) {
+  extern __shared__ __align__(16) float osm[];
+  float* xs = osm;                   // [kOneShotK][BT]
+  float* ws = osm + kOneShotK * BT;  // [kOneShotK][BE]
+  const int tid = threadIdx.x;
+  const int t0 = blockIdx.x * BT;
+  const int split = blockIdx.y;
+  const int k0 = split * kOneShotK;
+  const int row = tid & 127, h = tid >> 7;
+  const bool x_ok = (t0 + row) < T;
+  const bool w_ok = row < E;
+  const uint16_t* xrow = x + (size_t)(x_ok ? t0 + row : 0) * d + k0;
+  const float* wrow = wg + (size_t)(w_ok ? row : 0) * d + k0;
+  // every load first: 8 bf16 of x per uint4 (q = h + 2i of 8), 4 floats of
+  // w_gate per float4 (q = h + 2i of 16)
+  uint4 xv[4];
+  float4 wv[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    xv[i] = x_ok ? *reinterpret_cast<const uint4*>(xrow + (h + 2 * i) * 8) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    wv[i] = w_ok ? *reinterpret_cast<const float4*>(wrow + (h + 2 * i) * 4)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int kb = (h + 2 * i) * 8;
+    const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      xs[(kb + 2 * j) * BT + row] = bf16_bits_to_float(xw[j] & 0xFFFFu);
+      xs[(kb + 2 * j + 1) * BT + row] = bf16_bits_to_float(xw[j] >> 16);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int kb = (h + 2 * i) * 4;
+    ws[(kb + 0) * BE + row] = wv[i].x;
+    ws[(kb + 1) * BE + row] = wv[i].y;
+    ws[(kb + 2) * BE + row] = wv[i].z;
+    ws[(kb + 3) * BE + row] = wv[i].w;
+  }
+  __syncthreads();
+
+  const int ty = tid >> 4, tx = tid & 15;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+#pragma unroll 8
+  for (int kk = 0; kk < kOneShotK; ++kk) {
+    const float4 a0 = *reinterpret_cast<const float4*>(&xs[kk * BT + ty * 4]);
+    const float4 a1 = *reinterpret_cast<const float4*>(&xs[kk * BT + 64 + ty * 4]);
+    const float4 b0 = *reinterpret_cast<const float4*>(&ws[kk * BE + tx * 4]);
+    const float4 b1 = *reinterpret_cast<const float4*>(&ws[kk * BE + 64 + tx * 4]);
+    const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+  }
+
+  float* out = part + (size_t)split * T * E;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int t = t0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
+    if (t >= T) continue;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int e0 = half * 64 + tx * 4;
+      float* dst = out + (size_t)t * E + e0;
+      if (e0 + 3 < E && (E & 3) == 0) {
+        *reinterpret_cast<float4*>(dst) = make_float4(acc[i][half * 4 + 0], acc[i][half * 4 + 1],
+                                                      acc[i][half * 4 + 2], acc[i][half * 4 + 3]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (e0 + j < E) dst[j] = acc[i][half * 4 + j];
+      }
+    }
+  }
+}
+
 struct Cand {
   float key;
   int e;
@@ -298,8 +393,17 @@ cudaError_t launch_router(const Shape& s, const uint16_t* x, const float* w_gate
   if (s.T == 0) return cudaSuccess;
   const SplitPlan sp = plan_splits(s, num_sms);
   dim3 grid((unsigned)ceil_div(s.T, BT), (unsigned)sp.splits);
-  router_gemm_kernel<<<grid, kThreads, 0, st>>>(x, w_gate, partials, s.T, s.d, s.E, sp.kchunk);
-  cudaError_t err = cudaGetLastError();
+  cudaError_t err;
+  if (grid.x == 1 && sp.kchunk == kOneShotK && (int64_t)sp.splits * kOneShotK == s.d) {
+    err = cudaFuncSetAttribute(router_gemm_oneshot_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kOneShotSmem);
+    if (err != cudaSuccess) return err;
+    router_gemm_oneshot_kernel<<<grid, kThreads, kOneShotSmem, st>>>(x, w_gate, partials, s.T,
+                                                                     s.d, s.E);
+  } else {
+    router_gemm_kernel<<<grid, kThreads, 0, st>>>(x, w_gate, partials, s.T, s.d, s.E, sp.kchunk);
+  }
+  err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   router_topk_kernel<<<(unsigned)ceil_div(s.T, kTopkWarps), kTopkWarps * 32, 0, st>>>(
       partials, sp.splits, bias, probs, topk_idx, topk_w, s.T, s.E, s.k);
