@@ -324,9 +324,10 @@ def run_ours(args):
                "P": torch.empty((T // seq_len, cfg.E), **f32), "loss": torch.empty(1, **f32)}
         bias_next = torch.empty_like(layer.bias)
 
-        def step(xin, yout, evs=None):
+        def step(xin, yout, evs=None, dyin=None, dxout=None):
             layer.forward_train(xin, yout)
-            layer.backward(xin, dy, grads)
+            g = grads if dxout is None else dict(grads, dx=dxout)
+            layer.backward(xin, dy if dyin is None else dyin, g)
             if evs is not None:
                 evs[0].record(stream)
             layer.balance_stats(T, seq_len, BALANCE_ALPHA, out=bal)
@@ -334,7 +335,7 @@ def run_ours(args):
             if evs is not None:
                 evs[1].record(stream)
     else:
-        def step(xin, yout, evs=None):
+        def step(xin, yout, evs=None, dyin=None, dxout=None):
             layer(xin, yout)
     n_events = 13 if train else 6
     phase_names = M.PHASES + (M.BWD_PHASES if train else ())
@@ -349,9 +350,45 @@ def run_ours(args):
                               else layer.workspace(T))
     counts = views["counts"].cpu().numpy()
 
-    # ---- device-resident timed region (with per-phase events)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_events)]
-          for _ in range(args.steps)]
+    # ---- per-phase breakdown: an untimed pass with every phase bracketed
+    n_phase = min(args.steps, 20)
+    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_events)]
+           for _ in range(n_phase)]
+    bal_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+              for _ in range(n_phase)] if train else [None] * n_phase
+    for s in range(n_phase):
+        M.set_phase_events(pev[s])
+        step(x, y, bal_ev[s])
+    torch.cuda.synchronize(dev)
+    M.set_phase_events(None)
+    phase_ms = {}
+    bracket = {}  # phase -> (event before, event after) in the hook's list
+    for i, name in enumerate(M.PHASES):
+        bracket[name] = (i, i + 1)
+    for i, name in enumerate(M.BWD_PHASES if train else ()):
+        bracket[name] = (6 + i, 7 + i)
+    for name, (a, b) in bracket.items():
+        phase_ms[name] = statistics.mean(pev[s][a].elapsed_time(pev[s][b])
+                                         for s in range(n_phase))
+    if train:
+        phase_ms["balance_stats_bias_step"] = statistics.mean(
+            bal_ev[s][0].elapsed_time(bal_ev[s][1]) for s in range(n_phase))
+    units = gemm_units(cfg, T, counts)
+    if train:
+        tflops = train_gemm_flops(cfg, T)
+        dom = max(tflops, key=lambda n: phase_ms[n])
+    else:
+        dom = max(("gemm_gate_up_swiglu", "gemm_down"), key=lambda n: phase_ms[n])
+
+    # ---- device-resident timed region: only the dominant kernel's two
+    # bounding events are recorded, so the hook costs the step nothing else
+    ia, ib = bracket[dom]
+    ev = []
+    for _ in range(args.steps):
+        row = [None] * n_events
+        row[ia] = torch.cuda.Event(enable_timing=True)
+        row[ib] = torch.cuda.Event(enable_timing=True)
+        ev.append(row)
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
@@ -361,11 +398,9 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     t0 = time.time()
     start.record(stream)
-    bal_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
-              for _ in range(args.steps)] if train else [None] * args.steps
     for s in range(args.steps):
         M.set_phase_events(ev[s])
-        step(x, y, bal_ev[s])
+        step(x, y)
     end.record(stream)
     torch.cuda.synchronize(dev)
     t1 = time.time()
@@ -379,61 +414,73 @@ def run_ours(args):
     ms_local = start.elapsed_time(end)
     ms = max_over_ranks(ms_local, world, dev)
     value = whole_job_value(world, T, args.steps, ms)
-    phase_ms = {}
-    for i, name in enumerate(M.PHASES):
-        phase_ms[name] = statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1])
-                                         for s in range(args.steps))
-    for i, name in enumerate(M.BWD_PHASES if train else ()):
-        phase_ms[name] = statistics.mean(ev[s][6 + i].elapsed_time(ev[s][7 + i])
-                                         for s in range(args.steps))
-    if train:
-        phase_ms["balance_stats_bias_step"] = statistics.mean(
-            bal_ev[s][0].elapsed_time(bal_ev[s][1]) for s in range(args.steps))
+    dom_ms = statistics.mean(ev[s][ia].elapsed_time(ev[s][ib]) for s in range(args.steps))
 
-    # ---- end to end through the public API: pinned host x -> y on host
+    # ---- end to end through the public API: every step copies its inputs
+    # from pinned host memory and reads its result back.  The copies run on
+    # their own streams with double-buffered device tensors, so step i's
+    # copies overlap the neighbouring steps' compute (as a serving loop
+    # would); each step still moves all of its bytes inside the timed region.
+    h2d_st = torch.cuda.Stream(dev)
+    d2h_st = torch.cuda.Stream(dev)
     x_host = x.cpu().pin_memory()
-    y_host = torch.empty((T, cfg.d), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(x)
+    out_host = [torch.empty((T, cfg.d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    x_buf = [torch.empty_like(x) for _ in range(2)]
+    y_buf = [torch.empty_like(y) for _ in range(2)]
     if train:
         dy_host = dy.cpu().pin_memory()
-        dy_dev = dy
+        dy_buf = [torch.empty_like(dy) for _ in range(2)]
+        dx_buf = [torch.empty_like(grads["dx"]) for _ in range(2)]
+    in_ready = [torch.cuda.Event() for _ in range(2)]   # inputs of buffer b on the device
+    computed = [torch.cuda.Event() for _ in range(2)]   # the step using buffer b is done
+    out_read = [torch.cuda.Event() for _ in range(2)]   # result of buffer b read back
 
-        def e2e_step():
-            x_dev.copy_(x_host, non_blocking=True)
-            dy_dev.copy_(dy_host, non_blocking=True)
-            step(x_dev, y)
-            y_host.copy_(grads["dx"], non_blocking=True)
-    else:
-        def e2e_step():
-            x_dev.copy_(x_host, non_blocking=True)
-            step(x_dev, y)
-            y_host.copy_(y, non_blocking=True)
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
+    def e2e_step(i):
+        b = i & 1
+        h2d_st.wait_event(computed[b])   # the step that last used buffer b has finished
+        with torch.cuda.stream(h2d_st):
+            x_buf[b].copy_(x_host, non_blocking=True)
+            if train:
+                dy_buf[b].copy_(dy_host, non_blocking=True)
+        in_ready[b].record(h2d_st)
+        stream.wait_event(in_ready[b])
+        stream.wait_event(out_read[b])   # its previous result has been read out
+        if train:
+            step(x_buf[b], y_buf[b], dyin=dy_buf[b], dxout=dx_buf[b])
+        else:
+            step(x_buf[b], y_buf[b])
+        computed[b].record(stream)
+        d2h_st.wait_event(computed[b])
+        with torch.cuda.stream(d2h_st):
+            out_host[b].copy_(dx_buf[b] if train else y_buf[b], non_blocking=True)
+        out_read[b].record(d2h_st)
+
+    for i in range(max(1, args.warmup)):
+        e2e_step(i)
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    h2d_st.wait_event(e0)
+    d2h_st.wait_event(e0)
+    for i in range(args.steps):
+        e2e_step(i)
+    stream.wait_event(out_read[0])
+    stream.wait_event(out_read[1])
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = whole_job_value(world, T, args.steps, e2e_ms)
 
-    # ---- roofline of the dominant kernel
+    # ---- roofline of the dominant kernel (its duration from the timed region)
     peaks, peak_src = load_peaks()
-    units = gemm_units(cfg, T, counts)
     if train:
-        tflops = train_gemm_flops(cfg, T)
-        dom = max(tflops, key=lambda n: phase_ms[n])
         bytes_, flops = 0, tflops[dom]
     else:
-        dom = max(("gemm_gate_up_swiglu", "gemm_down"), key=lambda n: phase_ms[n])
         bytes_, flops = units[dom]
-    dur_s = phase_ms[dom] / 1e3
+    dur_s = dom_ms / 1e3
     hbm_bound = (not train) and T * cfg.k <= 24 * cfg.E
     if hbm_bound:
         achieved = bytes_ / dur_s / 1e9
@@ -461,6 +508,8 @@ def run_ours(args):
                          f"({(units['touched_experts'] + cfg.S) * 3 * cfg.I * cfg.d * 2 / 1e9:.2f} GB)"},
         "roofline": roof,
         "phases_ms": {k: round(v, 4) for k, v in phase_ms.items()},
+        "phases_ms_source": f"untimed pass of {n_phase} steps with every phase bracketed by "
+                            "events; the timed region brackets only the roofline kernel",
         "clocks": clocks,
         "e2e": {"value": e2e_value, "unit": "tokens/s",
                 "h2d_bytes_per_step": T * cfg.d * 2 * (2 if train else 1),

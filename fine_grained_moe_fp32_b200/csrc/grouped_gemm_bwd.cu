@@ -587,7 +587,8 @@ cudaError_t launch_backward_gemms(const Shape& s, const BackwardGemmArgs& a, int
   if (!small && pair_backward_supported(s))
     return launch_backward_gemms_pair(s, a, num_sms, status, wait_ns, st, events);
   auto mark = [&](int i) {
-    return events != nullptr ? cudaEventRecord(events[i], st) : cudaSuccess;
+    return events != nullptr && events[i] != nullptr ? cudaEventRecord(events[i], st)
+                                                     : cudaSuccess;
   };
   const bool shared = s.S > 0 && s.T > 0;
   const int SI = s.S * s.I;

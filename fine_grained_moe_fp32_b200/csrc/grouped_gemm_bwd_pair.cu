@@ -713,7 +713,8 @@ cudaError_t launch_backward_gemms_pair(const Shape& s, const BackwardGemmArgs& a
                                        unsigned int* status, uint64_t wait_ns, cudaStream_t st,
                                        const cudaEvent_t* events) {
   auto mark = [&](int i) {
-    return events != nullptr ? cudaEventRecord(events[i], st) : cudaSuccess;
+    return events != nullptr && events[i] != nullptr ? cudaEventRecord(events[i], st)
+                                                     : cudaSuccess;
   };
   const bool shared = s.S > 0;
   const int SI = s.S * s.I;

@@ -22,12 +22,15 @@ cudaEvent_t g_phase_events[kAllEvents] = {};
 bool g_phase_on = false;       // forward events set
 bool g_bwd_phase_on = false;   // backward events set too
 
+// A null entry of the event list is a point the caller does not time.
 cudaError_t phase(int i, cudaStream_t st) {
-  return g_phase_on ? cudaEventRecord(g_phase_events[i], st) : cudaSuccess;
+  return g_phase_on && g_phase_events[i] != nullptr ? cudaEventRecord(g_phase_events[i], st)
+                                                     : cudaSuccess;
 }
 
 cudaError_t bwd_phase(int i, cudaStream_t st) {
-  return g_bwd_phase_on ? cudaEventRecord(g_phase_events[kFwdEvents + i], st) : cudaSuccess;
+  cudaEvent_t e = g_phase_events[kFwdEvents + i];
+  return g_bwd_phase_on && e != nullptr ? cudaEventRecord(e, st) : cudaSuccess;
 }
 
 struct DeviceInfo {
@@ -536,10 +539,7 @@ int moe_set_phase_events(void* const* events, int n) {
     return MOE_OK;
   }
   if (n != kFwdEvents && n != kAllEvents) return MOE_ERR_INVALID_ARG;
-  for (int i = 0; i < n; ++i) {
-    if (events[i] == nullptr) return MOE_ERR_INVALID_ARG;
-    g_phase_events[i] = static_cast<cudaEvent_t>(events[i]);
-  }
+  for (int i = 0; i < n; ++i) g_phase_events[i] = static_cast<cudaEvent_t>(events[i]);
   g_phase_on = true;
   g_bwd_phase_on = n == kAllEvents;
   return MOE_OK;

@@ -346,14 +346,16 @@ def set_phase_events(events) -> None:
     """Record torch.cuda.Event objects between the kernels of moe_forward
     (6 events: before the router, then after each of the 5 phases) and, with
     13 events, of moe_backward too (before it, then after each of its 6
-    phases); None turns the hook off."""
+    phases); None turns the hook off.  An entry may be None: that point is
+    not recorded (timing one phase needs only its two bounding events)."""
     if events is None:
         _check(load().moe_set_phase_events(None, 0), "moe_set_phase_events")
         return
     for e in events:
-        if e.cuda_event == 0:   # torch creates the CUDA event on first record
+        if e is not None and e.cuda_event == 0:   # torch creates the event on first record
             e.record()
-    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    arr = (ctypes.c_void_p * len(events))(
+        *[ctypes.c_void_p(e.cuda_event if e is not None else None) for e in events])
     _check(load().moe_set_phase_events(arr, len(events)), "moe_set_phase_events")
 
 

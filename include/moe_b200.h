@@ -347,9 +347,11 @@ int moe_set_wait_limit_ns(uint64_t ns);
  * GEMM and the combine, on its stream.  With n == 13, moe_backward also
  * records events[6] before its first kernel and events[7..12] after the
  * combine/router backward, the dH + SwiGLU-backward dgrad, the dW2 wgrad, the
- * dX dgrad, the dW1/dW3 wgrads and the gate GEMMs + un-permute.  n == 0 (or
- * events == NULL) turns the hook off.  Process-wide; the events must outlive
- * every call issued while they are set.
+ * dX dgrad, the dW1/dW3 wgrads and the gate GEMMs + un-permute.  An entry may
+ * be NULL: that point is not recorded (timing one phase needs only its two
+ * bounding events, which keeps the hook's own cost out of the others).
+ * n == 0 (or events == NULL) turns the hook off.  Process-wide; the events
+ * must outlive every call issued while they are set.
  * ---------------------------------------------------------------------- */
 int moe_set_phase_events(void* const* events, int n);
 
