@@ -256,26 +256,38 @@ __device__ __forceinline__ bool better(const Cand& a, const Cand& b) {
 
 constexpr int kTopkWarps = 8;
 
+// WPT warps per token: warp q sums the contiguous run of split partials
+// [q * per, (q + 1) * per) in fp64 in ascending order (the loads of 16 splits
+// issued together so their latencies overlap), the runs are added in q order
+// through shared memory, and the token's first warp does softmax and top-k.
+// Many splits (decode) use 8 warps per token so each warp needs one round of
+// loads; a few splits (prefill) use one.
+template <int WPT>
 __global__ void __launch_bounds__(kTopkWarps * 32)
 router_topk_kernel(const float* __restrict__ part, int splits, const float* __restrict__ bias,
                    float* __restrict__ probs, int32_t* __restrict__ topk_idx,
                    float* __restrict__ topk_w, int T, int E, int k) {
+  constexpr int kTok = kTopkWarps / WPT;  // tokens per CTA
+  __shared__ double red[WPT > 1 ? kTopkWarps : 1][WPT > 1 ? 128 : 1];
   const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kTopkWarps + (threadIdx.x >> 5);
-  if (t >= T) return;
+  const int warp = threadIdx.x >> 5;
+  const int q = warp % WPT;
+  const int t = blockIdx.x * kTok + warp / WPT;
+  const bool live = t < T;
 
   bool valid[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) valid[i] = lane + 32 * i < E;
-  // split partials summed in fp64 in ascending split order; the loads of 16
-  // splits are issued together so their latencies overlap
+  const int per = (splits + WPT - 1) / WPT;
+  const int sp_begin = q * per;
+  const int sp_end = min(splits, sp_begin + per);
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
   constexpr int kU = 16;
-  for (int sp0 = 0; sp0 < splits; sp0 += kU) {
+  for (int sp0 = sp_begin; live && sp0 < sp_end; sp0 += kU) {
     float v[kU][4];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      const int sp = min(sp0 + u, splits - 1);  // clamped: every load is in bounds
+      const int sp = min(sp0 + u, sp_end - 1);  // clamped: every load is in bounds
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         v[u][i] = __ldg(part + ((size_t)sp * T + t) * E + min(lane + 32 * i, E - 1));
@@ -284,8 +296,21 @@ router_topk_kernel(const float* __restrict__ part, int splits, const float* __re
     for (int u = 0; u < kU; ++u)
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        if (sp0 + u < splits) acc[i] += (double)v[u][i];
+        if (sp0 + u < sp_end) acc[i] += (double)v[u][i];
   }
+  if constexpr (WPT > 1) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) red[warp][lane + 32 * i] = acc[i];
+    __syncthreads();
+    if (q != 0) return;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[i] = red[warp][lane + 32 * i];
+#pragma unroll
+      for (int r = 1; r < WPT; ++r) acc[i] += red[warp + r][lane + 32 * i];
+    }
+  }
+  if (!live) return;
   float z[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) z[i] = valid[i] ? (float)acc[i] : -INFINITY;
@@ -405,8 +430,18 @@ cudaError_t launch_router(const Shape& s, const uint16_t* x, const float* w_gate
   }
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  router_topk_kernel<<<(unsigned)ceil_div(s.T, kTopkWarps), kTopkWarps * 32, 0, st>>>(
-      partials, sp.splits, bias, probs, topk_idx, topk_w, s.T, s.E, s.k);
+  auto topk = [&](auto kern, int wpt) {
+    kern<<<(unsigned)ceil_div(s.T, kTopkWarps / wpt), kTopkWarps * 32, 0, st>>>(
+        partials, sp.splits, bias, probs, topk_idx, topk_w, s.T, s.E, s.k);
+  };
+  if (sp.splits > 64)
+    topk(router_topk_kernel<8>, 8);
+  else if (sp.splits > 32)
+    topk(router_topk_kernel<4>, 4);
+  else if (sp.splits > 16)
+    topk(router_topk_kernel<2>, 2);
+  else
+    topk(router_topk_kernel<1>, 1);
   return cudaGetLastError();
 }
 

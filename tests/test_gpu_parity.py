@@ -72,6 +72,9 @@ ROUTE_CASES = [
     ("E8_k1", MoEConfig("e8k1", T=77, d=128, E=8, k=1, S=1, I=64, bias="uniform0.01"), None),
     ("E128_k8", MoEConfig("k8", T=129, d=384, E=128, k=8, S=2, I=64, bias="normal0.05"), None),
     ("decode_full", CONFIGS[1], None),
+    # 46 and 18 split partials: the top-k sums them with 4 and 2 warps per token
+    ("d5120_T300_46_splits", CONFIGS[1], 300),
+    ("d5120_T1024_18_splits", CONFIGS[2], 1024),
     ("skewed_zipf_slice", CONFIGS[3], 2048),
 ]
 
