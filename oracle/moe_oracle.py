@@ -182,6 +182,13 @@ def swiglu_expert(xr, w1, w3, w2):
     return h @ _f64(w2).T, h, g, u
 
 
+def dense_swiglu(x, w1, w3, w2) -> np.ndarray:
+    """The dense SwiGLU FFN of the model's first layer (Technical Report,
+    Method: layer 1 is a dense SwiGLU FFN, the other layers MoE):
+    y = (silu(x W1^T) * (x W3^T)) W2^T on every token."""
+    return swiglu_expert(x, w1, w3, w2)[0]
+
+
 # --------------------------------------------------------------------------
 # Whole layer
 # --------------------------------------------------------------------------

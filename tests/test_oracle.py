@@ -228,6 +228,19 @@ def test_single_expert_is_textbook_ffn():
     np.testing.assert_allclose(f["y"], F0 + Fs, rtol=1e-10, atol=1e-12)
 
 
+def test_dense_swiglu_is_textbook_ffn_and_one_expert_layer():
+    """The dense layer equals torch's textbook SwiGLU FFN, and equals the MoE
+    layer reduced to one routed expert (k = 1, weight 1) with no shared one."""
+    cfg = MoEConfig("e1s0", T=12, d=32, E=1, k=1, S=0, I=24)
+    inp = make_inputs(cfg)
+    inp = {k: (v.double().numpy() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    y = O.dense_swiglu(inp["x"], inp["w1"][0], inp["w3"][0], inp["w2"][0])
+    np.testing.assert_allclose(
+        y, _dense_ffn_torch(inp["x"], inp["w1"][0], inp["w3"][0], inp["w2"][0]),
+        rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(y, O.forward(inp, align=4)["y"], rtol=1e-12, atol=1e-14)
+
+
 # ---------------------------------------------------------------- whole layer
 
 def test_dense_mask_brute_force_tiny_config():
