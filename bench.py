@@ -535,6 +535,137 @@ def run_ours(args):
     return 0
 
 
+DENSE_METRIC = "dense SwiGLU FFN tokens/s (bf16, d=5120, I=11264) and % of roofline"
+
+
+def run_dense(args):
+    """The first layer's dense SwiGLU FFN (moe_dense_swiglu) on the workload's
+    token count: device-resident timing, roofline, pipelined end-to-end copies."""
+    from fine_grained_moe_fp32_b200 import moe as M
+    from fine_grained_moe_fp32_b200.workloads import DENSE_I, make_dense_inputs
+    world, rank, local = dist_setup()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    T = args.tokens or CONFIGS[args.config].T
+    d = CONFIGS[args.config].d
+    I = args.inter or DENSE_I
+    inp = make_dense_inputs(T, d, I, device=dev, seed=shard_seed(0, rank) if world > 1 else 0)
+    dm = M.dense_dims(T, d, I)
+    ws = M.alloc_workspace(M.dense_workspace_size(dm), dev)
+    x, w1, w3, w2 = inp["x"], inp["w1"], inp["w3"], inp["w2"]
+    y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(xin, yout):
+        M.dense_swiglu(dm, xin, w1, w3, w2, yout, ws)
+
+    for _ in range(args.warmup):
+        step(x, y)
+    torch.cuda.synchronize(dev)
+    if M.device_status() != M.MOE_OK:
+        raise SystemExit("device status after warm-up")
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    time.sleep(0.15)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t0 = time.time()
+    start.record(stream)
+    for _ in range(args.steps):
+        step(x, y)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    t1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop(t0, t1)
+    if M.device_status() != M.MOE_OK:
+        raise SystemExit("device status after timing")
+    ms = max_over_ranks(start.elapsed_time(end), world, dev)
+    value = whole_job_value(world, T, args.steps, ms)
+
+    # end to end: x in from pinned memory, y back, on copy streams (double-buffered)
+    h2d_st, d2h_st = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    x_host = x.cpu().pin_memory()
+    y_host = [torch.empty((T, d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    xb = [torch.empty_like(x) for _ in range(2)]
+    yb = [torch.empty_like(y) for _ in range(2)]
+    ready = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    read = [torch.cuda.Event() for _ in range(2)]
+
+    def e2e_step(i):
+        b = i & 1
+        h2d_st.wait_event(done[b])
+        with torch.cuda.stream(h2d_st):
+            xb[b].copy_(x_host, non_blocking=True)
+        ready[b].record(h2d_st)
+        stream.wait_event(ready[b])
+        stream.wait_event(read[b])
+        step(xb[b], yb[b])
+        done[b].record(stream)
+        d2h_st.wait_event(done[b])
+        with torch.cuda.stream(d2h_st):
+            y_host[b].copy_(yb[b], non_blocking=True)
+        read[b].record(d2h_st)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    h2d_st.wait_event(e0)
+    d2h_st.wait_event(e0)
+    for i in range(args.steps):
+        e2e_step(i)
+    stream.wait_event(read[0])
+    stream.wait_event(read[1])
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_value = whole_job_value(world, T, args.steps, max_over_ranks(e0.elapsed_time(e1), world, dev))
+
+    peaks, peak_src = load_peaks()
+    dur_s = ms / args.steps / 1e3
+    flops = 2.0 * T * d * I * 3
+    bytes_ = 3.0 * I * d * 2 + 2.0 * T * d * 2 + T * I * 2 * 2
+    # bound by whichever floor is longer: streaming the weights or the flops
+    hbm_bound = bytes_ / (peaks["hbm_gbs"] * 1e9) >= flops / (peaks["bf16_tflops"] * 1e12)
+    if hbm_bound:
+        ach = bytes_ / dur_s / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"]}
+    else:
+        ach = flops / dur_s / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"]}
+    roof.update({"kernel": "dense step (gate/up + down grouped GEMMs as one group)",
+                 "peak_source": peak_src, "traffic": None,
+                 "algorithmic_per_launch": bytes_ if hbm_bound else flops})
+    if rank == 0:
+        print(json.dumps({
+            "metric": DENSE_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights)",
+            "config": {"workload": f"dense_swiglu_T{T}_d{d}_I{I}", "T": T, "d": d, "I": I,
+                       "parallelism": f"dp{world} (replicas, no collective)"},
+            "roofline": roof, "clocks": clocks,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
+                    "d2h_bytes_per_step": T * d * 2},
+            "gpu_launches": 3 * args.steps}), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[1])
     ap.add_argument("--gpus", type=int, default=1)
@@ -549,11 +680,15 @@ def main(argv=None):
     ap.add_argument("--experts", type=int, default=0, help="shrink E (profiling cases)")
     ap.add_argument("--tokens", type=int, default=0, help="override T (profiling cases)")
     ap.add_argument("--inter", type=int, default=0, help="override I (profiling cases)")
+    ap.add_argument("--dense", action="store_true",
+                    help="time the first layer's dense SwiGLU FFN instead of the MoE layer")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.dense:
+        return run_dense(args)
     return run_ours(args)
 
 

@@ -481,6 +481,74 @@ int moe_backward(const moe_dims* dims, const moe_bf16* x, const float* w_gate, c
   return cuda_status(e);
 }
 
+}  // extern "C"
+
+namespace moe {
+namespace {
+
+// The dense FFN runs the grouped GEMMs as one group holding every token.
+__global__ void dense_offsets_kernel(int32_t* offsets, int T) {
+  offsets[0] = 0;
+  offsets[1] = T;
+}
+
+int dense_shape(const moe_dims* dims, Shape* s) {
+  if (dims == nullptr || dims->T < 0 || dims->d <= 0 || dims->I <= 0) return MOE_ERR_INVALID_ARG;
+  if (dims->d % 128 != 0 || dims->I % 64 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if ((int64_t)dims->T * dims->I >= INT32_MAX / 2 || (int64_t)dims->T * dims->d >= INT32_MAX / 2)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  // capacity = T: the token operand is x itself, and its tensor map must not
+  // claim rows past the caller's T (tiles read zeros beyond it)
+  *s = Shape{dims->T, dims->d, 1, 1, dims->I, 0, 16, (int64_t)dims->T};
+  return MOE_OK;
+}
+
+size_t dense_h_offset() { return al256(2 * sizeof(int32_t)); }
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+size_t moe_dense_workspace_size(const moe_dims* dims) {
+  Shape s;
+  if (dense_shape(dims, &s) != MOE_OK) return 0;
+  return dense_h_offset() + al256((size_t)s.T * s.I * 2);
+}
+
+int moe_dense_swiglu(const moe_dims* dims, const moe_bf16* x, const moe_bf16* w1,
+                     const moe_bf16* w3, const moe_bf16* w2, moe_bf16* y, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = dense_shape(dims, &s);
+  if (rc != MOE_OK) return rc;
+  if (s.T == 0) return MOE_OK;
+  if (x == nullptr || w1 == nullptr || w3 == nullptr || w2 == nullptr || y == nullptr ||
+      !aligned(x, 16) || !aligned(w1, 16) || !aligned(w3, 16) || !aligned(w2, 16) ||
+      !aligned(y, 16))
+    return MOE_ERR_INVALID_ARG;
+  if (workspace == nullptr || !aligned(workspace, 256) ||
+      workspace_bytes < moe_dense_workspace_size(dims))
+    return MOE_ERR_WORKSPACE;
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* offsets = at<int32_t>(workspace, 0);
+  dense_offsets_kernel<<<1, 1, 0, st>>>(offsets, s.T);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  GroupedGemmArgs a{};
+  a.x_perm = x;
+  a.offsets = offsets;
+  a.w1 = w1;
+  a.w3 = w3;
+  a.w2 = w2;
+  a.h_perm = at<uint16_t>(workspace, dense_h_offset());
+  a.y_perm = y;
+  return cuda_status(
+      launch_grouped_gemms(s, a, di->num_sms, di->status, g_wait_limit_ns, st, nullptr));
+}
+
 size_t moe_balance_workspace_size(const moe_dims* dims, int seq_len) {
   Shape s;
   if (check_dims(dims, &s) != MOE_OK || seq_len <= 0 || s.T % seq_len != 0) return 0;

@@ -29,6 +29,7 @@ EXPORTED = (
     "moe_set_wait_limit_ns", "moe_set_phase_events", "moe_route_noalloc",
     "moe_train_workspace_size", "moe_train_layout_of", "moe_forward_train", "moe_backward",
     "moe_balance_workspace_size", "moe_balance_stats", "moe_bias_update",
+    "moe_dense_workspace_size", "moe_dense_swiglu",
 )
 
 
@@ -93,6 +94,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_balance_workspace_size": (Z, [P, I]),
         "moe_balance_stats": (I, [P, I, V, V, ctypes.c_float, V, V, V, V, Z, V]),
         "moe_bias_update": (I, [P, V, ctypes.c_float, V, V, V]),
+        "moe_dense_workspace_size": (Z, [P]),
+        "moe_dense_swiglu": (I, [P, V, V, V, V, V, V, Z, V]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -298,6 +301,28 @@ def backward(dm, x, w_gate, w1, w3, w2, ws1, ws3, ws2, dy, workspace, grads: dic
                              _ptr(g["dw3"]), _ptr(g["dw2"]), _ptr(g.get("dws1")),
                              _ptr(g.get("dws3")), _ptr(g.get("dws2")), _stream(stream))
     _check(rc, "moe_backward")
+
+
+def dense_dims(T, d, I) -> MoeDims:
+    """Dims of the dense FFN (E, k, n_shared are not used by it)."""
+    return dims(T, d, 1, 1, I, 0)
+
+
+def dense_workspace_size(dm: MoeDims) -> int:
+    return int(load().moe_dense_workspace_size(ctypes.byref(dm)))
+
+
+def dense_swiglu(dm, x, w1, w3, w2, y, workspace, stream=None):
+    """y = (silu(x w1^T) * (x w3^T)) w2^T: the first layer's dense SwiGLU FFN."""
+    _expect(x, torch.bfloat16, (dm.T, dm.d), "x")
+    _expect(w1, torch.bfloat16, (dm.I, dm.d), "w1")
+    _expect(w3, torch.bfloat16, (dm.I, dm.d), "w3")
+    _expect(w2, torch.bfloat16, (dm.d, dm.I), "w2")
+    _expect(y, torch.bfloat16, (dm.T, dm.d), "y")
+    rc = load().moe_dense_swiglu(ctypes.byref(dm), _ptr(x), _ptr(w1), _ptr(w3), _ptr(w2),
+                                 _ptr(y), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "moe_dense_swiglu")
 
 
 def balance_workspace_size(dm: MoeDims, seq_len: int) -> int:

@@ -69,7 +69,13 @@ CONFIGS = {
 
 # one independent stream per tensor, so shrinking T leaves the weights alone
 _STREAM = {"x": 1, "w_gate": 2, "bias": 3, "w1": 4, "w3": 5, "w2": 6,
-           "ws1": 7, "ws3": 8, "ws2": 9, "dy": 10, "zipf_perm": 11}
+           "ws1": 7, "ws3": 8, "ws2": 9, "dy": 10, "zipf_perm": 11,
+           "dense_w1": 12, "dense_w3": 13, "dense_w2": 14}
+
+# The first layer's dense SwiGLU FFN: its intermediate size is not on the
+# pages; the MoE layer's activated width (6 routed + 2 shared experts of 1408)
+# is used, so both layers cost the same per token.
+DENSE_I = 8 * 1408
 
 
 def _gen(seed: int, name: str, device) -> torch.Generator:
@@ -134,6 +140,19 @@ def make_inputs(cfg: MoEConfig | int, device="cpu", seed: int = 0,
     if cfg.grad:
         out["dy"] = _normal((T, d), 1.0, seed, "dy", dev, torch.bfloat16)
     return out
+
+
+def make_dense_inputs(T: int, d: int = 5120, I: int = DENSE_I, device="cpu",
+                      seed: int = 0) -> dict:
+    """Tokens and weights of the dense SwiGLU FFN: x N(0,1) bf16 [T, d];
+    w1, w3 [I, d] and w2 [d, I] N(0, 0.02) bf16.  x is the same draw as the
+    MoE workloads' x for the same (seed, T, d)."""
+    dev = torch.device(device)
+    return {"T": T, "d": d, "I": I,
+            "x": _normal((T, d), 1.0, seed, "x", dev, torch.bfloat16),
+            "w1": _normal((I, d), 0.02, seed, "dense_w1", dev, torch.bfloat16),
+            "w3": _normal((I, d), 0.02, seed, "dense_w3", dev, torch.bfloat16),
+            "w2": _normal((d, I), 0.02, seed, "dense_w2", dev, torch.bfloat16)}
 
 
 def small_config(T=64, d=256, E=16, k=4, S=2, I=128, bias="uniform0.01") -> MoEConfig:

@@ -279,6 +279,27 @@ int moe_backward(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
                  void* stream);
 
 /* ------------------------------------------------------------------------
+ * moe_dense_swiglu -- the dense SwiGLU FFN of the model's first layer
+ * (Technical Report, Method: layer 1 is a dense SwiGLU FFN, layers 2-62 are
+ * MoE).  Runs on the same grouped GEMM kernels as the experts, as one group
+ * holding every token:
+ *
+ *   y = (silu(x w1^T) * (x w3^T)) w2^T
+ *
+ *   dims       T, d and I (the FFN's intermediate size) are used; E, k,
+ *              n_shared and align are ignored.  d % 128 == 0, I % 64 == 0.
+ *   x  [T, d]  bf16;  w1, w3 [I, d], w2 [d, I] bf16
+ *   y  [T, d]  bf16 out (h rounded to bf16, fp32 accumulation, one rounding)
+ *   workspace  moe_dense_workspace_size() bytes, 256-byte aligned (h [T, I]).
+ * Returns INVALID_ARG (null or misaligned pointer), UNSUPPORTED_SHAPE,
+ * WORKSPACE, CUDA.  T == 0 is a no-op.
+ * ---------------------------------------------------------------------- */
+size_t moe_dense_workspace_size(const moe_dims* dims);
+int moe_dense_swiglu(const moe_dims* dims, const moe_bf16* x, const moe_bf16* w1,
+                     const moe_bf16* w3, const moe_bf16* w2, moe_bf16* y,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Load balancing, training side.  Technical Report, Method: the router is
  * balanced by the DeepSeek auxiliary-loss-free per-expert bias, stepped after
  * each batch from the experts' loads, plus a sequence-wise balance loss

@@ -117,6 +117,21 @@ def test_balance_calls_rejected_on_host(lib):
         M.MOE_ERR_INVALID_ARG
 
 
+def test_dense_calls_rejected_on_host(lib):
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: every call below fails first
+    bad_d = M.dense_dims(T=16, d=200, I=128)
+    assert lib.moe_dense_workspace_size(ctypes.byref(bad_d)) == 0
+    assert lib.moe_dense_swiglu(ctypes.byref(bad_d), fake, fake, fake, fake, fake, fake, 1 << 30,
+                                None) == M.MOE_ERR_UNSUPPORTED_SHAPE
+    dm = M.dense_dims(T=16, d=256, I=128)
+    need = lib.moe_dense_workspace_size(ctypes.byref(dm))
+    assert need >= 16 * 128 * 2
+    assert lib.moe_dense_swiglu(ctypes.byref(dm), None, fake, fake, fake, fake, fake, need,
+                                None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_dense_swiglu(ctypes.byref(dm), fake, fake, fake, fake, fake, fake, 64,
+                                None) == M.MOE_ERR_WORKSPACE
+
+
 def test_status_strings(lib):
     for s in (0, -1, -2, -3, -4, -5):
         assert M.status_string(s) != "unknown status"
