@@ -324,14 +324,18 @@ def run_ours(args):
                "P": torch.empty((T // seq_len, cfg.E), **f32), "loss": torch.empty(1, **f32)}
         bias_next = torch.empty_like(layer.bias)
 
+        group = torch.distributed.group.WORLD if world > 1 else None
+
         def step(xin, yout, evs=None, dyin=None, dxout=None):
             layer.forward_train(xin, yout)
             g = grads if dxout is None else dict(grads, dx=dxout)
             layer.backward(xin, dy if dyin is None else dyin, g)
+            if world > 1:   # data parallel: sum the weight gradients of all replicas
+                M.allreduce_grads(g, group)
             if evs is not None:
                 evs[0].record(stream)
             layer.balance_stats(T, seq_len, BALANCE_ALPHA, out=bal)
-            layer.bias_step(T, BALANCE_GAMMA, out=bias_next)
+            layer.bias_step(T, BALANCE_GAMMA, out=bias_next, group=group)
             if evs is not None:
                 evs[1].record(stream)
     else:
@@ -519,7 +523,11 @@ def run_ours(args):
     }
     if train:
         line["config"]["step"] = ("forward (training, keeps g/u) + backward + sequence-wise "
-                                  f"balance statistics (seq_len {seq_len}) + bias step")
+                                  f"balance statistics (seq_len {seq_len}) + bias step"
+                                  + (" + weight-gradient all-reduce and summed expert loads "
+                                     "(NCCL)" if world > 1 else ""))
+        if world > 1:
+            line["config"]["parallelism"] = f"dp{world} (weight gradients all-reduced)"
         line["train_tflop_per_step"] = sum(train_gemm_flops(cfg, T).values()) / 1e12
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n, dt = oracle_sample(inp, args.cpu_tokens)

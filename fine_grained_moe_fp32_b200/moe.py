@@ -455,6 +455,22 @@ def global_loads(counts: torch.Tensor, T: int, group=None):
     return c, int(n.item())
 
 
+WEIGHT_GRADS = ("dw_gate", "dw1", "dw3", "dw2", "dws1", "dws3", "dws2")
+
+
+def allreduce_grads(grads: dict, group=None) -> dict:
+    """Data-parallel training: sum the weight gradients of every replica in
+    place (the input gradient dx stays per replica).  One collective per
+    tensor, in a fixed order on every rank; the caller scales by 1/world if
+    it wants the mean."""
+    import torch.distributed as dist
+    for name in WEIGHT_GRADS:
+        t = grads.get(name)
+        if t is not None and t.numel() > 0:
+            dist.all_reduce(t, group=group)
+    return grads
+
+
 class MoELayer:
     """The layer with its weights resident on one device; ``__call__`` runs
     moe_forward into a reusable workspace."""

@@ -111,3 +111,34 @@ def test_two_rank_bias_step_uses_global_loads_on_gloo():
         assert res[r]["c_all"] == res[r]["c_whole"]
         assert res[r]["step"] == res[r]["step_whole"]
     assert res[0]["step"] == res[1]["step"]      # every replica takes the same step
+
+
+def _grads_worker(rank, world, port, out):
+    """Every replica's weight gradients are summed; dx stays per replica."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    from fine_grained_moe_fp32_b200 import moe as M
+
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        g = {name: torch.full((3, 4), float(rank + 1)) for name in M.WEIGHT_GRADS}
+        g["dx"] = torch.full((2, 4), float(rank + 1))
+        M.allreduce_grads(g)
+        out[rank] = {"weights": [float(g[n].max()) for n in M.WEIGHT_GRADS] +
+                     [float(g[n].min()) for n in M.WEIGHT_GRADS],
+                     "dx": float(g["dx"].max())}
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_weight_gradient_allreduce_on_gloo():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.start_processes(_grads_worker, args=(world, port, out), nprocs=world, join=True,
+                           start_method="spawn")
+        res = dict(out)
+    for r in range(world):
+        assert all(v == 3.0 for v in res[r]["weights"])   # 1 + 2 on every rank
+        assert res[r]["dx"] == float(r + 1)
