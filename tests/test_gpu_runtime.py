@@ -51,3 +51,40 @@ def test_phase_events_cover_the_step():
     parts = [ev[i].elapsed_time(ev[i + 1]) for i in range(5)]
     assert all(p >= 0 for p in parts)
     assert sum(parts) <= outer[0].elapsed_time(outer[1]) * 1.01 + 0.05
+
+
+@pytest.mark.parametrize("cid,T", [(0, None), (1, None), (2, 1024)],
+                         ids=["tiny", "decode", "prefill_T1024_cta_pairs"])
+def test_forward_captures_into_a_cuda_graph(cid, T):
+    """moe_forward issues only stream work (no host sync, no allocation), so it
+    can be captured once and replayed: every replay gives the eager result bit
+    for bit, and a replay follows new input values written in place."""
+    import torch
+    from fine_grained_moe_fp32_b200 import moe as M
+    from fine_grained_moe_fp32_b200.workloads import CONFIGS, make_inputs
+    cfg = CONFIGS[cid]
+    inp = make_inputs(cfg, device="cuda", T=T)
+    layer = M.MoELayer(inp)
+    x = inp["x"].clone()
+    y = torch.empty((x.shape[0], cfg.d), dtype=torch.bfloat16, device="cuda")
+    eager = layer(x).clone()
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(st):
+        layer(x, y, stream=st)          # warm-up on the capture stream
+        st.synchronize()
+        with torch.cuda.graph(g, stream=st):
+            layer(x, y, stream=st)
+    torch.cuda.current_stream().wait_stream(st)
+    for _ in range(3):
+        y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), eager.view(torch.int16))
+    x2 = make_inputs(cfg, device="cuda", T=T, seed=5, weights=False)["x"]
+    x.copy_(x2)
+    g.replay()
+    torch.cuda.synchronize()
+    assert M.device_status() == M.MOE_OK
+    assert torch.equal(y.view(torch.int16), layer(x2).view(torch.int16))
