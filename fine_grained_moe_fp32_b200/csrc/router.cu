@@ -101,7 +101,9 @@ router_gemm_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wg,
   for (int kc = 0; kc < nk; ++kc) {
     const int buf = kc & 1;
     if (kc + 1 < nk) gload(kc + 1);
-#pragma unroll
+    // unrolled by 4, not fully: measured 15-25 % faster (the fully unrolled
+    // chunk at 255 registers issues worse); the arithmetic order is the same
+#pragma unroll 4
     for (int kk = 0; kk < BK; ++kk) {
       const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][kk][ty * 4]);
       const float4 a1 = *reinterpret_cast<const float4*>(&xs[buf][kk][64 + ty * 4]);
