@@ -438,3 +438,76 @@ def bias_update(bias, counts, gamma: float, T: int, k: int) -> np.ndarray:
     excess = E * c - T * k                 # E * (count - mean), exact integers
     step = -np.sign(excess).astype(np.float64)
     return np.where(step == 0, b, b + gamma * step)
+
+
+# --------------------------------------------------------------------------
+# Expert parallelism (Technical Report, Method / Key claims, systems
+# paragraph: the MoE all-to-all between ranks, overlapped with the grouped
+# GEMMs; "How dots.llm1's 14B MoE Architecture Matches 72B LLM Performance",
+# Computational Infrastructure Innovations: all-to-all expert communication).
+# The pages name the exchange but not its layout.  The reading used here:
+# rank r of W owns the experts [r E/W, (r+1) E/W); every rank routes its own
+# tokens; on the owner, expert e's segment holds the (token, slot) pairs of e
+# from every rank, ordered by source rank and then by the source's own
+# segment order (ascending token id), padded to `align` rows.  The layer's
+# output is unchanged by the exchange: each rank's y is forward() of its own
+# tokens.
+# --------------------------------------------------------------------------
+
+def ep_layout(idx_per_rank, E: int, align: int) -> dict:
+    """Receive layout of the dispatch among W = len(idx_per_rank) ranks.
+
+    idx_per_rank[s] is the [T_s, k] expert choice of rank s.  Returns
+
+      recv_offsets[r]  [E/W + 1]  first row of each local expert's segment on
+                                  rank r (segment le holds expert r E/W + le)
+      recv_counts[r]   [E/W]      pairs rank r receives for each local expert
+      owner[s], row[s] [T_s * k]  rank and receive row of pair (t, j) of rank s
+                                  at index t*k + j
+      src_of_row[r]    list of (source rank, token) per receive row of rank r,
+                       (-1, -1) for padding rows
+
+    Built by walking the pairs in the order the layout defines, one row at a
+    time.
+    """
+    W = len(idx_per_rank)
+    assert W > 0 and E % W == 0, "the experts must split evenly over the ranks"
+    El = E // W
+    idx = [np.asarray(a, dtype=np.int64) for a in idx_per_rank]
+    owner = [np.full(a.size, -1, dtype=np.int64) for a in idx]
+    row = [np.full(a.size, -1, dtype=np.int64) for a in idx]
+    recv_offsets = np.zeros((W, El + 1), dtype=np.int64)
+    recv_counts = np.zeros((W, El), dtype=np.int64)
+    src_of_row = []
+    for r in range(W):
+        rows = []
+        for le in range(El):
+            e = r * El + le
+            recv_offsets[r, le] = len(rows)
+            for s in range(W):
+                T_s, k = idx[s].shape
+                for t in range(T_s):
+                    for j in range(k):
+                        if idx[s][t, j] == e:
+                            owner[s][t * k + j] = r
+                            row[s][t * k + j] = len(rows)
+                            rows.append((s, t))
+            recv_counts[r, le] = len(rows) - recv_offsets[r, le]
+            while (len(rows) - recv_offsets[r, le]) % align:
+                rows.append((-1, -1))
+        recv_offsets[r, El] = len(rows)
+        src_of_row.append(rows)
+    return {"recv_offsets": recv_offsets, "recv_counts": recv_counts, "owner": owner,
+            "row": row, "src_of_row": src_of_row}
+
+
+def ep_recv_rows(x_per_rank, layout: dict, r: int) -> np.ndarray:
+    """Rows rank r holds after the dispatch: x of the source token of each
+    receive row, zero rows for padding."""
+    rows = layout["src_of_row"][r]
+    d = _f64(x_per_rank[0][:1]).shape[1]
+    out = np.zeros((len(rows), d))
+    for i, (s, t) in enumerate(rows):
+        if s >= 0:
+            out[i] = _f64(x_per_rank[s][t:t + 1])[0]
+    return out

@@ -475,3 +475,83 @@ def test_bias_update_direction_and_fixed_point():
     np.testing.assert_allclose(np.abs(nb - bias)[nb != bias], gamma, rtol=1e-12)
     assert np.signbit(nb[2])
     np.testing.assert_array_equal(O.bias_update(bias, np.full(E, mean), gamma, T, k), bias)
+
+
+# ---- expert-parallel layout ------------------------------------------------
+
+def test_ep_layout_hand_example():
+    """W = 2 ranks, E = 4 experts (rank 0 owns 0-1, rank 1 owns 2-3), k = 2,
+    align = 2.  Rank 0 routes t0 -> {0, 1}, t1 -> {1, 3}; rank 1 routes
+    t0 -> {3, 0}, t1 -> {1, 2}.  Worked by hand: rank 0's expert 0 gets
+    (s0 t0), (s1 t0) = rows 0-1; expert 1 gets (s0 t0), (s0 t1), (s1 t1) =
+    rows 2-4 and one padding row 5.  Rank 1's expert 2 gets (s1 t1) = row 0 and
+    padding row 1; expert 3 gets (s0 t1), (s1 t0) = rows 2-3."""
+    L = O.ep_layout([np.array([[0, 1], [1, 3]]), np.array([[3, 0], [1, 2]])], 4, 2)
+    assert L["recv_offsets"].tolist() == [[0, 2, 6], [0, 2, 4]]
+    assert L["recv_counts"].tolist() == [[2, 3], [1, 2]]
+    assert L["owner"][0].tolist() == [0, 0, 0, 1] and L["row"][0].tolist() == [0, 2, 3, 2]
+    assert L["owner"][1].tolist() == [1, 0, 0, 1] and L["row"][1].tolist() == [3, 1, 4, 0]
+    assert L["src_of_row"][0] == [(0, 0), (1, 0), (0, 0), (0, 1), (1, 1), (-1, -1)]
+    assert L["src_of_row"][1] == [(1, 1), (-1, -1), (0, 1), (1, 0)]
+
+
+@pytest.mark.parametrize("align", [1, 16])
+def test_ep_layout_one_rank_is_the_permutation(align):
+    """With one rank the exchange is the identity: the receive layout is the
+    permutation's own segment layout."""
+    rng = np.random.default_rng(5)
+    idx = np.stack([rng.permutation(16)[:4] for _ in range(37)])
+    L = O.ep_layout([idx], 16, align)
+    P = O.permute(idx, 16, align)
+    assert L["recv_offsets"][0].tolist() == P["offsets"].tolist()
+    assert L["recv_counts"][0].tolist() == P["counts"].tolist()
+    assert L["row"][0].tolist() == P["row_of"].tolist()
+    assert (L["owner"][0] == 0).all()
+    tor = [t for (_, t) in L["src_of_row"][0]]
+    assert tor == P["token_of_row"][:len(tor)].tolist()
+
+
+@pytest.mark.parametrize("W,E,k,align", [(2, 16, 4, 16), (4, 32, 3, 4), (8, 8, 2, 16)])
+def test_ep_layout_invariants_random_routing(W, E, k, align):
+    """Every pair lands exactly once, on the rank that owns its expert, inside
+    that expert's segment; segments are padded multiples of align and hold
+    the pairs by ascending (source rank, token); the ranks' loads add up."""
+    rng = np.random.default_rng(W * 100 + E)
+    T = [int(rng.integers(0, 40)) for _ in range(W)]
+    idx = [np.stack([rng.permutation(E)[:k] for _ in range(t)]) if t else
+           np.zeros((0, k), np.int64) for t in T]
+    L = O.ep_layout(idx, E, align)
+    El = E // W
+    taken = [set() for _ in range(W)]
+    for s in range(W):
+        for p in range(T[s] * k):
+            e = int(idx[s].reshape(-1)[p])
+            r, row = int(L["owner"][s][p]), int(L["row"][s][p])
+            assert r == e // El
+            le = e - r * El
+            assert L["recv_offsets"][r, le] <= row < L["recv_offsets"][r, le] + L["recv_counts"][r, le]
+            assert row not in taken[r]
+            taken[r].add(row)
+            assert L["src_of_row"][r][row] == (s, p // k)
+    for r in range(W):
+        off, cnt = L["recv_offsets"][r], L["recv_counts"][r]
+        assert off[0] == 0 and (np.diff(off) % align == 0).all()
+        assert (np.diff(off) >= cnt).all() and (np.diff(off) - cnt < align).all()
+        assert len(taken[r]) == cnt.sum()
+        for le in range(El):
+            seg = L["src_of_row"][r][off[le]:off[le] + cnt[le]]
+            assert seg == sorted(seg)                       # (source, token) ascending
+            assert all(s < 0 for s, _ in L["src_of_row"][r][off[le] + cnt[le]:off[le + 1]])
+    total = sum(int(L["recv_counts"][r].sum()) for r in range(W))
+    assert total == sum(T) * k
+
+
+def test_ep_recv_rows_gathers_the_source_tokens():
+    rng = np.random.default_rng(9)
+    x = [rng.standard_normal((5, 8)), rng.standard_normal((3, 8))]
+    idx = [np.array([[0, 1], [2, 3], [1, 2], [0, 3], [3, 1]]), np.array([[2, 0], [1, 3], [0, 2]])]
+    L = O.ep_layout(idx, 4, 4)
+    for r in range(2):
+        rows = O.ep_recv_rows(x, L, r)
+        for i, (s, t) in enumerate(L["src_of_row"][r]):
+            np.testing.assert_array_equal(rows[i], x[s][t] if s >= 0 else np.zeros(8))
