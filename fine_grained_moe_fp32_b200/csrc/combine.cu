@@ -1,6 +1,8 @@
 // Combine: weighted un-permute of the routed expert outputs plus the shared
 // experts (dots.llm1 Technical Report, Method: shared experts are always on;
-// the routed experts enter with their gate weights).
+// the routed experts enter with their gate weights).  With expert parallelism
+// the routed rows are read from the receive buffers of the ranks that own the
+// experts (the return half of the all-to-all, fused into the sum).
 //
 //   y[t] = y_shared[t] + sum_{j < k} w[t, j] * y_perm[row_of[t*k + j]]
 //
@@ -26,16 +28,42 @@ __device__ __forceinline__ void add_bf16x8(float (&acc)[8], uint4 v, float w) {
   }
 }
 
+// Where slot j of token t lives: its row of this rank's segment buffer.
+struct LocalRows {
+  const uint16_t* y_perm;
+  const int32_t* row_of;
+  int64_t cap;
+  __device__ const uint16_t* row(size_t p, int d) const {
+    const int r = row_of[p];
+    return (r >= 0 && r < cap) ? y_perm + (size_t)r * d : nullptr;
+  }
+};
+
+// Expert parallel: the row the dispatch wrote into the owner's receive
+// buffer, read back from there (peer loads when the owner is another GPU).
+struct OwnerRows {
+  const uint16_t* const* y_recv;
+  const int32_t* topk_idx;
+  const int32_t* remote_row;
+  int E, El;
+  int64_t cap;
+  __device__ const uint16_t* row(size_t p, int d) const {
+    const int e = topk_idx[p], r = remote_row[p];
+    if (e < 0 || e >= E || r < 0 || r >= cap) return nullptr;
+    const uint16_t* b = y_recv[e / El];
+    return (reinterpret_cast<uintptr_t>(b) & 15) ? nullptr : b + (size_t)r * d;
+  }
+};
+
+template <typename Rows>
 __global__ void __launch_bounds__(kThreads)
-combine_kernel(const uint16_t* __restrict__ y_perm, const int32_t* __restrict__ row_of,
-               const float* __restrict__ topk_w, const float* __restrict__ y_shared,
-               uint16_t* __restrict__ y, int d, int k, int64_t cap) {
+combine_kernel(Rows src, const float* __restrict__ topk_w, const float* __restrict__ y_shared,
+               uint16_t* __restrict__ y, int d, int k) {
   const int t = blockIdx.x;
-  __shared__ int rows[kMaxK];
+  __shared__ const uint16_t* rows[kMaxK];
   __shared__ float ws[kMaxK];
   if (threadIdx.x < k) {
-    const int r = row_of[(size_t)t * k + threadIdx.x];
-    rows[threadIdx.x] = (r >= 0 && r < cap) ? r : -1;
+    rows[threadIdx.x] = src.row((size_t)t * k + threadIdx.x, d);
     ws[threadIdx.x] = topk_w[(size_t)t * k + threadIdx.x];
   }
   __syncthreads();
@@ -55,11 +83,10 @@ combine_kernel(const uint16_t* __restrict__ y_perm, const int32_t* __restrict__ 
     uint4 val[kMaxK];
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j)
-      if (j < k && rows[j] >= 0)
-        val[j] = reinterpret_cast<const uint4*>(y_perm + (size_t)rows[j] * d)[v];
+      if (j < k && rows[j] != nullptr) val[j] = __ldg(reinterpret_cast<const uint4*>(rows[j]) + v);
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j)
-      if (j < k && rows[j] >= 0) add_bf16x8(acc, val[j], ws[j]);
+      if (j < k && rows[j] != nullptr) add_bf16x8(acc, val[j], ws[j]);
     uint32_t o[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -78,7 +105,19 @@ cudaError_t launch_combine(const Shape& s, const uint16_t* y_perm, const int32_t
                            cudaStream_t st) {
   if (s.T == 0) return cudaSuccess;
   const dim3 grid((unsigned)s.T, (unsigned)ceil_div(s.d / 8, kThreads));
-  combine_kernel<<<grid, kThreads, 0, st>>>(y_perm, row_of, topk_w, y_shared, y, s.d, s.k, s.cap);
+  combine_kernel<<<grid, kThreads, 0, st>>>(LocalRows{y_perm, row_of, s.cap}, topk_w, y_shared, y,
+                                            s.d, s.k);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ep_combine(const Shape& s, int world, const uint16_t* const* y_recv,
+                              const int32_t* topk_idx, const int32_t* remote_row, int64_t cap,
+                              const float* topk_w, const float* y_shared, uint16_t* y,
+                              cudaStream_t st) {
+  if (s.T == 0) return cudaSuccess;
+  const dim3 grid((unsigned)s.T, (unsigned)ceil_div(s.d / 8, kThreads));
+  const OwnerRows src{y_recv, topk_idx, remote_row, s.E, s.E / world, cap};
+  combine_kernel<<<grid, kThreads, 0, st>>>(src, topk_w, y_shared, y, s.d, s.k);
   return cudaGetLastError();
 }
 

@@ -583,6 +583,193 @@ int moe_bias_update(const moe_dims* dims, const int32_t* counts, float gamma,
       launch_bias_update(s, counts, gamma, bias_in, bias_out, static_cast<cudaStream_t>(stream)));
 }
 
+}  // extern "C"
+
+namespace moe {
+namespace {
+
+// Expert parallelism: the rank's own shape plus the receive capacity.
+int check_ep(const moe_dims* dims, int world, Shape* s, int64_t* rcap) {
+  int rc = check_dims(dims, s);
+  if (rc != MOE_OK) return rc;
+  if (world <= 0 || world > s->E || s->E % world != 0) return MOE_ERR_INVALID_ARG;
+  *rcap = ep_recv_capacity(*s, world);
+  if (*rcap >= (int64_t)INT32_MAX / 2) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+moe_ep_layout make_ep_layout(const Shape& s, int world, int64_t rcap) {
+  moe_ep_layout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += al256(bytes);
+    return at;
+  };
+  const int El = s.E / world;
+  L.route_partials = take(router_partials_bytes(s, kPlanSMs));
+  L.probs = take((size_t)s.T * s.E * 4);
+  L.topk_idx = take((size_t)s.T * s.k * 4);
+  L.topk_w = take((size_t)s.T * s.k * 4);
+  L.counts = take((size_t)s.E * 4);
+  L.offsets = take((size_t)(s.E + 1) * 4);
+  L.row_of = take((size_t)s.T * s.k * 4);
+  L.token_of_row = take((size_t)s.cap * 4);
+  L.permute_scratch = take(permute_scratch_bytes(s));
+  L.dst_row = take((size_t)s.E * 4);
+  L.recv_offsets = take((size_t)(El + 1) * 4);
+  L.recv_counts = take((size_t)El * 4);
+  L.remote_row = take((size_t)s.T * s.k * 4);
+  L.h_recv = take((size_t)rcap * s.I * 2);
+  L.h_shared = take((size_t)s.T * s.S * s.I * 2);
+  L.y_shared = take((size_t)s.T * s.d * 4);
+  L.total = off;
+  return L;
+}
+
+// Shared prologue of the EP entries: shape and workspace checks.
+int ep_prologue(const moe_dims* dims, int world, void* workspace, size_t workspace_bytes,
+                Shape* s, int64_t* rcap, moe_ep_layout* L) {
+  int rc = check_ep(dims, world, s, rcap);
+  if (rc != MOE_OK) return rc;
+  *L = make_ep_layout(*s, world, *rcap);
+  if (workspace == nullptr || workspace_bytes < L->total || !aligned(workspace, 256))
+    return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+int64_t moe_ep_recv_capacity(const moe_dims* dims, int world) {
+  Shape s;
+  int64_t rcap = 0;
+  return check_ep(dims, world, &s, &rcap) == MOE_OK ? rcap : 0;
+}
+
+size_t moe_ep_workspace_size(const moe_dims* dims, int world) {
+  Shape s;
+  int64_t rcap = 0;
+  if (check_ep(dims, world, &s, &rcap) != MOE_OK) return 0;
+  return make_ep_layout(s, world, rcap).total;
+}
+
+int moe_ep_layout_of(const moe_dims* dims, int world, moe_ep_layout* layout) {
+  Shape s;
+  int64_t rcap = 0;
+  int rc = check_ep(dims, world, &s, &rcap);
+  if (rc != MOE_OK) return rc;
+  if (layout == nullptr) return MOE_ERR_INVALID_ARG;
+  *layout = make_ep_layout(s, world, rcap);
+  return MOE_OK;
+}
+
+int moe_ep_route(const moe_dims* dims, int world, const moe_bf16* x, const float* w_gate,
+                 const float* bias, void* workspace, size_t workspace_bytes, void* stream) {
+  Shape s;
+  int64_t rcap;
+  moe_ep_layout L;
+  int rc = ep_prologue(dims, world, workspace, workspace_bytes, &s, &rcap, &L);
+  if (rc != MOE_OK) return rc;
+  if (w_gate == nullptr || (s.T > 0 && x == nullptr) || !aligned(x, 16) || !aligned(w_gate, 16))
+    return MOE_ERR_INVALID_ARG;
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  cudaError_t e = launch_router(s, x, w_gate, bias, at<float>(ws, L.probs),
+                                at<int32_t>(ws, L.topk_idx), at<float>(ws, L.topk_w),
+                                at<float>(ws, L.route_partials), kPlanSMs, st);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  return cuda_status(launch_permute(s, at<int32_t>(ws, L.topk_idx), x, at<int32_t>(ws, L.counts),
+                                    at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.row_of),
+                                    at<int32_t>(ws, L.token_of_row), nullptr,
+                                    at<void>(ws, L.permute_scratch), di->status, st));
+}
+
+int moe_ep_dispatch(const moe_dims* dims, int world, int rank, const moe_bf16* x,
+                    const int32_t* const* counts_of, moe_bf16* const* x_recv, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  Shape s;
+  int64_t rcap;
+  moe_ep_layout L;
+  int rc = ep_prologue(dims, world, workspace, workspace_bytes, &s, &rcap, &L);
+  if (rc != MOE_OK) return rc;
+  if (rank < 0 || rank >= world || counts_of == nullptr || x_recv == nullptr ||
+      (s.T > 0 && x == nullptr) || !aligned(x, 16))
+    return MOE_ERR_INVALID_ARG;
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return MOE_ERR_CUDA;
+  void* ws = workspace;
+  return cuda_status(launch_ep_dispatch(
+      s, world, rank, x, at<int32_t>(ws, L.topk_idx), at<int32_t>(ws, L.row_of),
+      at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.counts), counts_of, x_recv,
+      at<int32_t>(ws, L.dst_row), at<int32_t>(ws, L.recv_offsets), at<int32_t>(ws, L.recv_counts),
+      at<int32_t>(ws, L.remote_row), di->status, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_ep_experts(const moe_dims* dims, int world, const moe_bf16* x, const moe_bf16* x_recv,
+                   const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
+                   const moe_bf16* ws1, const moe_bf16* ws3, const moe_bf16* ws2,
+                   moe_bf16* y_recv, void* workspace, size_t workspace_bytes, void* stream) {
+  Shape s;
+  int64_t rcap;
+  moe_ep_layout L;
+  int rc = ep_prologue(dims, world, workspace, workspace_bytes, &s, &rcap, &L);
+  if (rc != MOE_OK) return rc;
+  if (x_recv == nullptr || y_recv == nullptr || w1 == nullptr || w3 == nullptr ||
+      w2 == nullptr || (s.T > 0 && s.S > 0 && x == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (s.S > 0 && (ws1 == nullptr || ws3 == nullptr || ws2 == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(x_recv, 16) || !aligned(y_recv, 16) || !aligned(w1, 16) ||
+      !aligned(w3, 16) || !aligned(w2, 16) || !aligned(ws1, 16) || !aligned(ws3, 16) ||
+      !aligned(ws2, 16))
+    return MOE_ERR_INVALID_ARG;
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return MOE_ERR_CUDA;
+  // the local experts' grouped GEMMs: El groups over the receive buffer
+  const Shape se{s.T, s.d, s.E / world, s.k, s.I, s.S, s.align, rcap};
+  void* ws = workspace;
+  GroupedGemmArgs a{};
+  a.x_perm = x_recv;
+  a.offsets = at<int32_t>(ws, L.recv_offsets);
+  a.w1 = w1;
+  a.w3 = w3;
+  a.w2 = w2;
+  a.h_perm = at<uint16_t>(ws, L.h_recv);
+  a.y_perm = y_recv;
+  if (s.S > 0) {
+    a.x = x;
+    a.ws1 = ws1;
+    a.ws3 = ws3;
+    a.ws2 = ws2;
+    a.h_shared = at<uint16_t>(ws, L.h_shared);
+    a.y_shared = at<float>(ws, L.y_shared);
+  }
+  return cuda_status(launch_grouped_gemms(se, a, di->num_sms, di->status, g_wait_limit_ns,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int moe_ep_combine(const moe_dims* dims, int world, const moe_bf16* const* y_recv, moe_bf16* y,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+  Shape s;
+  int64_t rcap;
+  moe_ep_layout L;
+  int rc = ep_prologue(dims, world, workspace, workspace_bytes, &s, &rcap, &L);
+  if (rc != MOE_OK) return rc;
+  if (s.T == 0) return MOE_OK;
+  if (y_recv == nullptr || y == nullptr || !aligned(y, 16)) return MOE_ERR_INVALID_ARG;
+  if (device_info() == nullptr) return MOE_ERR_CUDA;
+  void* ws = workspace;
+  return cuda_status(launch_ep_combine(s, world, y_recv, at<int32_t>(ws, L.topk_idx),
+                                       at<int32_t>(ws, L.remote_row), rcap,
+                                       at<float>(ws, L.topk_w),
+                                       s.S > 0 ? at<float>(ws, L.y_shared) : nullptr, y,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 int moe_get_last_device_status(void* stream) {
   const DeviceInfo* di = device_info();
   if (di == nullptr) return MOE_ERR_CUDA;
@@ -596,6 +783,7 @@ int moe_get_last_device_status(void* stream) {
   switch (v) {
     case DEV_OK: return MOE_OK;
     case DEV_BAD_EXPERT_ID: return MOE_ERR_INVALID_ARG;
+    case DEV_BAD_EP_LAYOUT: return MOE_ERR_INVALID_ARG;
     case DEV_TIMEOUT: return MOE_ERR_TIMEOUT;
     default: return MOE_ERR_CUDA;
   }

@@ -13,6 +13,7 @@ enum DevStatus : unsigned int {
   DEV_OK = 0,
   DEV_BAD_EXPERT_ID = 1,
   DEV_TIMEOUT = 2,
+  DEV_BAD_EP_LAYOUT = 3,  // expert-parallel counts inconsistent or over capacity
 };
 
 __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -126,5 +127,21 @@ cudaError_t launch_bias_update(const Shape& s, const int32_t* counts, float gamm
 cudaError_t launch_combine(const Shape& s, const uint16_t* y_perm, const int32_t* row_of,
                            const float* topk_w, const float* y_shared, uint16_t* y,
                            cudaStream_t st);
+// expert parallel: rows pulled from the owners' receive buffers
+// y_recv[idx / (E/world)] at remote_row (rows < cap; -1 = skipped)
+cudaError_t launch_ep_combine(const Shape& s, int world, const uint16_t* const* y_recv,
+                              const int32_t* topk_idx, const int32_t* remote_row, int64_t cap,
+                              const float* topk_w, const float* y_shared, uint16_t* y,
+                              cudaStream_t st);
+
+// ---- expert parallelism (expert_parallel.cu)
+// rows of a rank's receive buffer: world*T*k + (E/world)*(align-1)
+int64_t ep_recv_capacity(const Shape& s, int world);
+cudaError_t launch_ep_dispatch(const Shape& s, int world, int rank, const uint16_t* x,
+                               const int32_t* topk_idx, const int32_t* row_of,
+                               const int32_t* offsets, const int32_t* counts,
+                               const int32_t* const* counts_of, uint16_t* const* x_recv,
+                               int32_t* dst_row, int32_t* recv_offsets, int32_t* recv_counts,
+                               int32_t* remote_row, unsigned int* status, cudaStream_t st);
 
 }  // namespace moe

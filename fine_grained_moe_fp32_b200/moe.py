@@ -30,6 +30,8 @@ EXPORTED = (
     "moe_train_workspace_size", "moe_train_layout_of", "moe_forward_train", "moe_backward",
     "moe_balance_workspace_size", "moe_balance_stats", "moe_bias_update",
     "moe_dense_workspace_size", "moe_dense_swiglu",
+    "moe_ep_recv_capacity", "moe_ep_workspace_size", "moe_ep_layout_of", "moe_ep_route",
+    "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine",
 )
 
 
@@ -50,6 +52,13 @@ class MoeTrainLayout(ctypes.Structure):
     _fields_ = [("fwd", MoeWsLayout)] + [(n, ctypes.c_size_t) for n in (
         "g_perm", "u_perm", "g_shared", "u_shared", "dy_perm", "dw", "dz", "dgu_perm",
         "dgu_shared", "dx_perm", "dx_shared", "dx_router", "dwg_partials", "total")]
+
+
+class MoeEpLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in (
+        "route_partials", "probs", "topk_idx", "topk_w", "counts", "offsets", "row_of",
+        "token_of_row", "permute_scratch", "dst_row", "recv_offsets", "recv_counts",
+        "remote_row", "h_recv", "h_shared", "y_shared", "total")]
 
 
 class MoEError(RuntimeError):
@@ -96,6 +105,13 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_bias_update": (I, [P, V, ctypes.c_float, V, V, V]),
         "moe_dense_workspace_size": (Z, [P]),
         "moe_dense_swiglu": (I, [P, V, V, V, V, V, V, Z, V]),
+        "moe_ep_recv_capacity": (ctypes.c_int64, [P, I]),
+        "moe_ep_workspace_size": (Z, [P, I]),
+        "moe_ep_layout_of": (I, [P, I, ctypes.POINTER(MoeEpLayout)]),
+        "moe_ep_route": (I, [P, I, V, V, V, V, Z, V]),
+        "moe_ep_dispatch": (I, [P, I, I, V, V, V, V, Z, V]),
+        "moe_ep_experts": (I, [P, I, V, V, V, V, V, V, V, V, V, V, Z, V]),
+        "moe_ep_combine": (I, [P, I, V, V, V, Z, V]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -351,6 +367,159 @@ def bias_update(dm, counts, gamma, bias_in, bias_out, stream=None):
     rc = load().moe_bias_update(ctypes.byref(dm), _ptr(counts), float(gamma), _ptr(bias_in),
                                 _ptr(bias_out), _stream(stream))
     _check(rc, "moe_bias_update")
+
+
+# ------------------------------------------------------------ expert parallel
+
+def ep_recv_capacity(dm: MoeDims, world: int) -> int:
+    return int(load().moe_ep_recv_capacity(ctypes.byref(dm), int(world)))
+
+
+def ep_workspace_size(dm: MoeDims, world: int) -> int:
+    return int(load().moe_ep_workspace_size(ctypes.byref(dm), int(world)))
+
+
+def ep_layout(dm: MoeDims, world: int) -> dict:
+    L = MoeEpLayout()
+    _check(load().moe_ep_layout_of(ctypes.byref(dm), int(world), ctypes.byref(L)),
+           "moe_ep_layout_of")
+    return {n: getattr(L, n) for n, _ in MoeEpLayout._fields_}
+
+
+def pointer_array(tensors, device) -> torch.Tensor:
+    """A device array of the tensors' device addresses (int64), the form the
+    expert-parallel calls take for per-rank buffers."""
+    for t in tensors:
+        _ptr(t)
+    return torch.tensor([t.data_ptr() for t in tensors], dtype=torch.int64, device=device)
+
+
+def ep_route(dm, world, x, w_gate, bias, workspace, stream=None):
+    _expect(x, torch.bfloat16, (dm.T, dm.d), "x")
+    _check(load().moe_ep_route(ctypes.byref(dm), int(world), _ptr(x), _ptr(w_gate), _ptr(bias),
+                               _ptr(workspace), workspace.numel(), _stream(stream)),
+           "moe_ep_route")
+
+
+def ep_dispatch(dm, world, rank, x, counts_of, x_recv, workspace, stream=None):
+    """counts_of, x_recv: pointer_array() of every rank's counts / receive buffer."""
+    _expect(x, torch.bfloat16, (dm.T, dm.d), "x")
+    _check(load().moe_ep_dispatch(ctypes.byref(dm), int(world), int(rank), _ptr(x),
+                                  _ptr(counts_of), _ptr(x_recv), _ptr(workspace),
+                                  workspace.numel(), _stream(stream)), "moe_ep_dispatch")
+
+
+def ep_experts(dm, world, x, x_recv, w1, w3, w2, ws1, ws3, ws2, y_recv, workspace, stream=None):
+    El, rc = dm.E // world, ep_recv_capacity(dm, world)
+    _expect(x_recv, torch.bfloat16, (rc, dm.d), "x_recv")
+    _expect(y_recv, torch.bfloat16, (rc, dm.d), "y_recv")
+    _expect(w1, torch.bfloat16, (El, dm.I, dm.d), "w1")
+    _expect(w2, torch.bfloat16, (El, dm.d, dm.I), "w2")
+    _check(load().moe_ep_experts(ctypes.byref(dm), int(world), _ptr(x), _ptr(x_recv), _ptr(w1),
+                                 _ptr(w3), _ptr(w2), _ptr(ws1), _ptr(ws3), _ptr(ws2),
+                                 _ptr(y_recv), _ptr(workspace), workspace.numel(),
+                                 _stream(stream)), "moe_ep_experts")
+
+
+def ep_combine(dm, world, y_recv, y, workspace, stream=None):
+    """y_recv: pointer_array() of every rank's expert-output buffer."""
+    _expect(y, torch.bfloat16, (dm.T, dm.d), "y")
+    _check(load().moe_ep_combine(ctypes.byref(dm), int(world), _ptr(y_recv), _ptr(y),
+                                 _ptr(workspace), workspace.numel(), _stream(stream)),
+           "moe_ep_combine")
+
+
+def ep_workspace_views(dm: MoeDims, world: int, ws: torch.Tensor) -> dict:
+    """Typed views of one rank's expert-parallel workspace."""
+    L = ep_layout(dm, world)
+    T, E, k, I = dm.T, dm.E, dm.k, dm.I
+    El, rc = E // world, ep_recv_capacity(dm, world)
+
+    def view(off, n, dtype, shape):
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        return ws[off:off + nbytes].view(dtype).view(*shape)
+
+    i32 = torch.int32
+    return {
+        "probs": view(L["probs"], T * E, torch.float32, (T, E)),
+        "topk_idx": view(L["topk_idx"], T * k, i32, (T, k)),
+        "topk_w": view(L["topk_w"], T * k, torch.float32, (T, k)),
+        "counts": view(L["counts"], E, i32, (E,)),
+        "offsets": view(L["offsets"], E + 1, i32, (E + 1,)),
+        "row_of": view(L["row_of"], T * k, i32, (T * k,)),
+        "dst_row": view(L["dst_row"], E, i32, (E,)),
+        "recv_offsets": view(L["recv_offsets"], El + 1, i32, (El + 1,)),
+        "recv_counts": view(L["recv_counts"], El, i32, (El,)),
+        "remote_row": view(L["remote_row"], T * k, i32, (T * k,)),
+        "h_recv": view(L["h_recv"], rc * I, torch.bfloat16, (rc, I)),
+    }
+
+
+class EPRanks:
+    """Expert parallelism over ``world`` ranks emulated by one process on one
+    device: rank r owns experts [r E/W, (r+1) E/W) (its weight slices are
+    views of the full tensors) and its own receive buffers; the cross-rank
+    arguments are arrays of this device's buffers instead of peer pointers.
+    Each step issues, rank after rank, the same calls a rank of a multi-GPU
+    job makes, with stream order standing in for the barriers between the
+    phases, so no kernel ever waits on another."""
+
+    def __init__(self, inputs: dict, world: int, T: int, align: int = 16, device="cuda"):
+        cfg = inputs["cfg"]
+        if cfg.E % world:
+            raise ValueError("the routed experts must split evenly over the ranks")
+        self.cfg, self.world, self.T, self.align = cfg, int(world), int(T), align
+        self.device = torch.device(device)
+        to = lambda t: t.to(self.device).contiguous()  # noqa: E731
+        self.w_gate, self.bias = to(inputs["w_gate"]), to(inputs["bias"])
+        w1, w3, w2 = to(inputs["w1"]), to(inputs["w3"]), to(inputs["w2"])
+        self.ws1, self.ws3, self.ws2 = to(inputs["ws1"]), to(inputs["ws3"]), to(inputs["ws2"])
+        El = cfg.E // world
+        self.experts = [(w1[r * El:(r + 1) * El], w3[r * El:(r + 1) * El],
+                         w2[r * El:(r + 1) * El]) for r in range(world)]
+        self.dm = dims(T, cfg.d, cfg.E, cfg.k, cfg.I, cfg.S, align)
+        self.recv_cap = ep_recv_capacity(self.dm, world)
+        nbytes = ep_workspace_size(self.dm, world)
+        self.ws = [alloc_workspace(nbytes, self.device) for _ in range(world)]
+        bf = dict(dtype=torch.bfloat16, device=self.device)
+        self.x_recv = [torch.empty((self.recv_cap, cfg.d), **bf) for _ in range(world)]
+        self.y_recv = [torch.empty((self.recv_cap, cfg.d), **bf) for _ in range(world)]
+        self.views = [ep_workspace_views(self.dm, world, w) for w in self.ws]
+        self.counts_of = pointer_array([v["counts"] for v in self.views], self.device)
+        self.x_recv_of = pointer_array(self.x_recv, self.device)
+        self.y_recv_of = pointer_array(self.y_recv, self.device)
+
+    def route(self, xs, stream=None):
+        for r in range(self.world):
+            ep_route(self.dm, self.world, xs[r], self.w_gate, self.bias, self.ws[r], stream)
+
+    def dispatch(self, xs, stream=None):
+        for r in range(self.world):
+            ep_dispatch(self.dm, self.world, r, xs[r], self.counts_of, self.x_recv_of, self.ws[r],
+                        stream)
+
+    def experts_step(self, xs, stream=None):
+        for r in range(self.world):
+            w1, w3, w2 = self.experts[r]
+            ep_experts(self.dm, self.world, xs[r], self.x_recv[r], w1, w3, w2, self.ws1,
+                       self.ws3, self.ws2, self.y_recv[r], self.ws[r], stream)
+
+    def combine(self, ys, stream=None):
+        for r in range(self.world):
+            ep_combine(self.dm, self.world, self.y_recv_of, ys[r], self.ws[r], stream)
+
+    def __call__(self, xs, ys=None, stream=None):
+        """xs: the ranks' token batches ([T, d] bf16 each); returns their y."""
+        if len(xs) != self.world:
+            raise ValueError(f"expected {self.world} token batches")
+        if ys is None:
+            ys = [torch.empty((self.T, self.cfg.d), dtype=torch.bfloat16, device=self.device)
+                  for _ in range(self.world)]
+        self.route(xs, stream)
+        self.dispatch(xs, stream)
+        self.experts_step(xs, stream)
+        self.combine(ys, stream)
+        return ys
 
 
 def device_status(stream=None) -> int:

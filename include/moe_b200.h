@@ -345,6 +345,114 @@ int moe_bias_update(const moe_dims* dims, const int32_t* counts, float gamma,
                     const float* bias_in, float* bias_out, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Expert parallelism.  Technical Report, Method / Key claims (systems
+ * paragraph): the MoE all-to-all between ranks, overlapped with the grouped
+ * GEMMs; "How dots.llm1's 14B MoE Architecture Matches 72B LLM Performance",
+ * Computational Infrastructure Innovations: all-to-all expert communication.
+ * The pages name the exchange, not its layout; the layout used:
+ *
+ *   world W ranks, every rank routes its own T tokens (same dims on every
+ *   rank); rank r owns the routed experts r*El .. r*El + El-1, El = E/W, and
+ *   holds only their weights; the shared experts are replicated and run on
+ *   each rank's own tokens.  Rank r's receive buffer holds one segment per
+ *   local expert, padded to `align` rows, with the (token, slot) pairs of
+ *   every source rank in rank order, each source's pairs by ascending token.
+ *   Every rank derives this layout from all ranks' counts, so a source writes
+ *   its token rows straight into the owners' receive buffers and the combine
+ *   reads the expert outputs back from them.
+ *
+ * A step on rank r, with barriers between ranks where marked:
+ *   moe_ep_route       router + permutation index of the own tokens
+ *   -- barrier (every rank's counts written) --
+ *   moe_ep_dispatch    layout from every rank's counts; each pair's token row
+ *                      stored into its owner's receive buffer; padding rows of
+ *                      the own receive buffer zeroed
+ *   -- barrier (every receive buffer complete) --
+ *   moe_ep_experts     grouped SwiGLU GEMMs of the El local experts over the
+ *                      receive buffer, and the shared experts on own tokens
+ *   -- barrier (every owner's outputs complete) --
+ *   moe_ep_combine     y[t] = shared + sum_j w[t,j] * (row of pair (t, j) in
+ *                      its owner's output buffer), fp32, j ascending, as
+ *                      moe_combine
+ * The barriers are the caller's (e.g. a one-element NCCL all-reduce on the
+ * same stream); the library waits on nothing.  Cross-rank arguments are
+ * DEVICE arrays of W device pointers, element s for rank s: peer pointers
+ * (CUDA IPC or a symmetric allocation) on a multi-GPU node, or plain buffers
+ * of this GPU when several ranks are emulated by one process.
+ *
+ * moe_ep_recv_capacity  rows of a receive buffer: W*T*k + El*(align-1)
+ *                       (0 on invalid arguments)
+ * moe_ep_workspace_size bytes of one rank's workspace; moe_ep_layout_of
+ *                       reports where its regions are:
+ */
+typedef struct moe_ep_layout {
+  size_t route_partials;  /* fp32 router split-K partials                   */
+  size_t probs;           /* fp32 [T, E]                                   */
+  size_t topk_idx;        /* int32 [T, k]                                  */
+  size_t topk_w;          /* fp32 [T, k]                                   */
+  size_t counts;          /* int32 [E]   own pairs per expert (peers read)  */
+  size_t offsets;         /* int32 [E+1] own segment layout                */
+  size_t row_of;          /* int32 [T*k]                                   */
+  size_t token_of_row;    /* int32 [T*k + E*(align-1)]                     */
+  size_t permute_scratch; /* permutation scratch                           */
+  size_t dst_row;         /* int32 [E]   first receive row of the own pairs
+                                         of expert e on its owner (-1 after
+                                         a rejected count table)           */
+  size_t recv_offsets;    /* int32 [El+1] segment starts in the own buffer  */
+  size_t recv_counts;     /* int32 [El]  pairs received per local expert    */
+  size_t remote_row;      /* int32 [T*k] receive row of pair (t, j), -1 if
+                                         not sent                          */
+  size_t h_recv;          /* bf16 [recv_cap, I] local experts' SwiGLU out   */
+  size_t h_shared;        /* bf16 [T, S*I]                                 */
+  size_t y_shared;        /* fp32 [T, d]                                   */
+  size_t total;           /* = moe_ep_workspace_size()                     */
+} moe_ep_layout;
+
+int64_t moe_ep_recv_capacity(const moe_dims* dims, int world);
+size_t moe_ep_workspace_size(const moe_dims* dims, int world);
+int moe_ep_layout_of(const moe_dims* dims, int world, moe_ep_layout* layout);
+
+/* moe_ep_route -- x [T, d] bf16, w_gate [E, d] fp32, bias [E] fp32 (NULL =
+ * zero): moe_route and the index half of moe_permute (no row gather) into
+ * the workspace.  Results equal theirs bit for bit. */
+int moe_ep_route(const moe_dims* dims, int world, const moe_bf16* x,
+                 const float* w_gate, const float* bias, void* workspace,
+                 size_t workspace_bytes, void* stream);
+
+/* moe_ep_dispatch --
+ *   counts_of  device array [W] of int32 [E] pointers: every rank's counts
+ *              (element s = rank s's workspace counts, or a gathered copy);
+ *              element `rank` must equal this rank's own counts
+ *   x_recv     device array [W] of bf16 [recv_cap, d] receive buffers,
+ *              16-byte aligned
+ * A count table that is negative, disagrees with the own counts or overflows
+ * a receive buffer is recorded as MOE_ERR_INVALID_ARG in the device status
+ * word and nothing is sent or received. */
+int moe_ep_dispatch(const moe_dims* dims, int world, int rank, const moe_bf16* x,
+                    const int32_t* const* counts_of, moe_bf16* const* x_recv,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* moe_ep_experts --
+ *   x        [T, d] bf16 own tokens (shared experts)
+ *   x_recv   [recv_cap, d] this rank's receive buffer
+ *   w1, w3   [El, I, d], w2 [El, d, I] bf16: this rank's experts only
+ *   ws1, ws3 [S, I, d], ws2 [S, d, I] shared experts (NULL iff S == 0)
+ *   y_recv   [recv_cap, d] bf16 out: expert outputs per receive row
+ * Rows at or after the last segment are neither read nor written. */
+int moe_ep_experts(const moe_dims* dims, int world, const moe_bf16* x,
+                   const moe_bf16* x_recv, const moe_bf16* w1, const moe_bf16* w3,
+                   const moe_bf16* w2, const moe_bf16* ws1, const moe_bf16* ws3,
+                   const moe_bf16* ws2, moe_bf16* y_recv, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
+/* moe_ep_combine --
+ *   y_recv  device array [W] of the ranks' expert-output buffers
+ *   y       [T, d] bf16 out
+ * Same arithmetic as moe_combine; a pair that was not sent contributes 0. */
+int moe_ep_combine(const moe_dims* dims, int world, const moe_bf16* const* y_recv,
+                   moe_bf16* y, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Device status and bounded waits.
  *
  * moe_get_last_device_status: synchronises `stream`, returns the first error

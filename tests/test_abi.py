@@ -132,6 +132,37 @@ def test_dense_calls_rejected_on_host(lib):
                                 None) == M.MOE_ERR_WORKSPACE
 
 
+def test_expert_parallel_sizes_and_rejects_on_host(lib):
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: every call below fails first
+    dm = M.dims(T=128, d=5120, E=128, k=6, I=1408, n_shared=2, align=16)
+    assert M.ep_recv_capacity(dm, 8) == 8 * 128 * 6 + 16 * 15
+    assert M.ep_recv_capacity(dm, 1) == M.capacity(dm)
+    for bad_world in (0, -1, 3, 129):
+        assert M.ep_recv_capacity(dm, bad_world) == 0
+        assert M.ep_workspace_size(dm, bad_world) == 0
+    L = M.ep_layout(dm, 8)
+    offs = [L[n] for n, _ in M.MoeEpLayout._fields_ if n != "total"]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert L["total"] == M.ep_workspace_size(dm, 8)
+    assert L["h_shared"] - L["h_recv"] >= M.ep_recv_capacity(dm, 8) * 1408 * 2
+    need = L["total"]
+    P = ctypes.byref(dm)
+    assert lib.moe_ep_route(P, 3, fake, fake, None, fake, need, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_route(P, 8, fake, fake, None, fake, 64, None) == M.MOE_ERR_WORKSPACE
+    assert lib.moe_ep_route(P, 8, None, fake, None, fake, need, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_dispatch(P, 8, 8, fake, fake, fake, fake, need, None) == \
+        M.MOE_ERR_INVALID_ARG                                       # rank out of range
+    assert lib.moe_ep_dispatch(P, 8, 0, fake, None, fake, fake, need, None) == \
+        M.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_experts(P, 8, fake, None, fake, fake, fake, fake, fake, fake, fake, fake,
+                              need, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_experts(P, 8, fake, fake, fake, fake, fake, None, fake, fake, fake, fake,
+                              need, None) == M.MOE_ERR_INVALID_ARG   # S = 2 without ws1
+    assert lib.moe_ep_combine(P, 8, None, fake, fake, need, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_combine(P, 8, fake, fake, ctypes.c_void_p((1 << 20) + 64), need,
+                              None) == M.MOE_ERR_WORKSPACE
+
+
 def test_status_strings(lib):
     for s in (0, -1, -2, -3, -4, -5):
         assert M.status_string(s) != "unknown status"
