@@ -674,6 +674,160 @@ def run_dense(args):
     return 0
 
 
+def ep_kernels(T: int) -> int:
+    """Launches of one emulated rank's expert-parallel step: router GEMM +
+    top-k, the permutation index (one kernel for at most 256 tokens, else
+    count, scan, scatter), the layout plan, the dispatch, the two grouped
+    GEMMs, the combine."""
+    return 2 + (1 if T <= 256 else 3) + 2 + 2 + 1
+
+
+def run_ep(args):
+    """Expert parallelism over --ep W ranks emulated on one GPU: each step
+    runs every rank's route, dispatch, expert GEMMs and combine (the calls a
+    rank of a multi-GPU job makes) on this device, stream order standing in
+    for the barriers.  Every rank routes its own batch of the workload's T
+    tokens; the value counts all W*T tokens."""
+    from fine_grained_moe_fp32_b200 import moe as M
+    world, rank, local = dist_setup()
+    if world > 1:
+        raise SystemExit("--ep emulates the ranks on one GPU; run it without torchrun")
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cfg = workload(args)
+    W, T = args.ep, cfg.T
+    inp = make_inputs(cfg, device=dev)
+    xs = [inp["x"]] + [make_inputs(cfg, device=dev, seed=1000 + r, weights=False)["x"]
+                       for r in range(1, W)]
+    ep = M.EPRanks(inp, W, T, args.align, dev)
+    ys = [torch.empty((T, cfg.d), dtype=torch.bfloat16, device=dev) for _ in range(W)]
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        ep(xs, ys)
+    torch.cuda.synchronize(dev)
+    if M.device_status() != M.MOE_OK:
+        raise SystemExit("device status after warm-up")
+
+    # phase pass (untimed): events between the four phases of every step
+    names = ("route", "dispatch", "experts", "combine")
+    n_phase = min(args.steps, 20)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_phase)]
+    for i in range(n_phase):
+        ev[i][0].record(stream)
+        ep.route(xs)
+        ev[i][1].record(stream)
+        ep.dispatch(xs)
+        ev[i][2].record(stream)
+        ep.experts_step(xs)
+        ev[i][3].record(stream)
+        ep.combine(ys)
+        ev[i][4].record(stream)
+    torch.cuda.synchronize(dev)
+    phase_ms = {n: statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(n_phase))
+                for j, n in enumerate(names)}
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    time.sleep(0.15)
+    torch.cuda.synchronize(dev)
+    t0 = time.time()
+    start.record(stream)
+    for _ in range(args.steps):
+        ep(xs, ys)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    t1 = time.time()
+    clocks = sampler.stop(t0, t1)
+    if M.device_status() != M.MOE_OK:
+        raise SystemExit("device status after timing")
+    ms = start.elapsed_time(end)
+    value = W * T * args.steps / (ms / 1e3)
+
+    # end to end through the same calls: every rank's x in from pinned host
+    # memory and its y back, inside the timed region
+    x_host = [x.cpu().pin_memory() for x in xs]
+    y_host = [torch.empty((T, cfg.d), dtype=torch.bfloat16).pin_memory() for _ in range(W)]
+    xb = [torch.empty_like(x) for x in xs]
+    for _ in range(args.warmup):
+        for r in range(W):
+            xb[r].copy_(x_host[r], non_blocking=True)
+        ep(xb, ys)
+        for r in range(W):
+            y_host[r].copy_(ys[r], non_blocking=True)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        for r in range(W):
+            xb[r].copy_(x_host[r], non_blocking=True)
+        ep(xb, ys)
+        for r in range(W):
+            y_host[r].copy_(ys[r], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_value = W * T * args.steps / (e0.elapsed_time(e1) / 1e3)
+
+    # algorithmic work per phase, from the routing of the last step
+    d, I, S, k = cfg.d, cfg.I, cfg.S, cfg.k
+    El = cfg.E // W
+    recv = [v["recv_counts"].cpu().numpy().astype(np.int64) for v in ep.views]
+    pad = [int(v["recv_offsets"][-1]) - int(c.sum()) for v, c in zip(ep.views, recv)]
+    exp_bytes = exp_flops = 0
+    for c in recv:
+        rows, touched = int(c.sum()), int((c > 0).sum())
+        exp_bytes += ((touched + S) * 3 * I * d * 2 + (rows + T) * d * 2
+                      + 2 * (rows + T * S) * I * 2 + rows * d * 2 + T * d * 4)
+        exp_flops += 2 * (rows * 3 * I + T * 3 * S * I) * d
+    disp_bytes = W * T * d * 2 + W * T * k * d * 2 + sum(pad) * d * 2
+    comb_bytes = W * (T * k * d * 2 + T * d * (4 if S else 0) + T * d * 2)
+    peaks, peak_src = load_peaks()
+    # bound by whichever floor is longer: streaming the bytes or the flops
+    hbm_bound = exp_bytes / (peaks["hbm_gbs"] * 1e9) >= exp_flops / (peaks["bf16_tflops"] * 1e12)
+    dur_s = phase_ms["experts"] / 1e3
+    if hbm_bound:
+        ach = exp_bytes / dur_s / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"]}
+    else:
+        ach = exp_flops / dur_s / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"]}
+    roof.update({"kernel": f"expert GEMMs of all {W} ranks (2 grouped GEMMs per rank)",
+                 "peak_source": f"{peak_src} ({'hbm_gbs' if hbm_bound else 'bf16_tflops'})",
+                 "traffic": None, "algorithmic_per_launch": exp_bytes if hbm_bound else exp_flops,
+                 "duration_source": "phase pass (events around the expert GEMMs of all ranks)"})
+    phases = {n: {"ms": round(phase_ms[n], 4)} for n in names}
+    phases["dispatch"]["GB/s"] = round(disp_bytes / (phase_ms["dispatch"] / 1e3) / 1e9, 1)
+    phases["combine"]["GB/s"] = round(comb_bytes / (phase_ms["combine"] / 1e3) / 1e9, 1)
+    line = {
+        "metric": METRIC + f"; expert parallel over {W} ranks emulated on one GPU",
+        "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) tokens per rank, N(0,0.02) weights; random-init layer)",
+        "config": {"workload": f"ep{W}_emulated_{cfg.name}", "ranks": W, "T_per_rank": T,
+                   "d": d, "E": cfg.E, "experts_per_rank": El, "k": k, "S": S, "I": I,
+                   "align": args.align, "recv_capacity_rows": ep.recv_cap,
+                   "parallelism": f"ep{W} emulated (one process, one GPU)",
+                   "l2": "inputs larger than L2: the step streams the expert weights"},
+        "roofline": roof, "phases": phases, "clocks": clocks,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": W * T * d * 2,
+                "d2h_bytes_per_step": W * T * d * 2},
+        "gpu_launches": W * ep_kernels(T) * args.steps,
+    }
+    if not args.no_cpu_baseline:
+        n, secs = oracle_sample(inp, args.cpu_tokens)
+        line["cpu_baseline"] = {"value": n / secs, "unit": "tokens/s", "cores": cpu_threads(),
+                                "kind": "oracle",
+                                "sample": f"{n} seeded tokens of rank 0's batch, fp64 numpy "
+                                          f"oracle (forward; the exchange does not change it), "
+                                          f"{secs:.1f} s"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[1])
     ap.add_argument("--gpus", type=int, default=1)
@@ -688,6 +842,8 @@ def main(argv=None):
     ap.add_argument("--experts", type=int, default=0, help="shrink E (profiling cases)")
     ap.add_argument("--tokens", type=int, default=0, help="override T (profiling cases)")
     ap.add_argument("--inter", type=int, default=0, help="override I (profiling cases)")
+    ap.add_argument("--ep", type=int, default=0,
+                    help="expert parallelism over this many ranks emulated on one GPU")
     ap.add_argument("--dense", action="store_true",
                     help="time the first layer's dense SwiGLU FFN instead of the MoE layer")
     args = ap.parse_args(argv)
@@ -697,6 +853,8 @@ def main(argv=None):
         return run_reference(args)
     if args.dense:
         return run_dense(args)
+    if args.ep:
+        return run_ep(args)
     return run_ours(args)
 
 
