@@ -67,6 +67,12 @@ CONFIGS = {
     4: MoEConfig("fwd_bwd_T8192_d5120_I1408", T=8192, d=5120, grad=True),
 }
 
+TINY = CONFIGS[0]
+DECODE = CONFIGS[1]
+PREFILL_BALANCED = CONFIGS[2]
+PREFILL_SKEWED = CONFIGS[3]
+FWD_BWD = CONFIGS[4]
+
 # one independent stream per tensor, so shrinking T leaves the weights alone
 _STREAM = {"x": 1, "w_gate": 2, "bias": 3, "w1": 4, "w3": 5, "w2": 6,
            "ws1": 7, "ws3": 8, "ws2": 9, "dy": 10, "zipf_perm": 11,

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from fine_grained_moe_fp32_b200 import moe as M
-from fine_grained_moe_fp32_b200.workloads import CONFIGS, MoEConfig, make_inputs, small_config
+from fine_grained_moe_fp32_b200.workloads import (CONFIGS, MoEConfig, make_inputs, small_config, FWD_BWD, TINY)
 from oracle import moe_oracle as O
 import parity_utils as PU
 
@@ -89,7 +89,7 @@ def _check_all(inp, y_inf, y, grads, f, b, experts=None, spec=True):
 
 
 CASES = [
-    ("tiny_full", CONFIGS[0], None),
+    ("tiny_full", TINY, None),
     ("small_E16_T200", small_config(T=200, d=256, E=16, k=4, I=128), None),
     ("E32_S1_k8_T97", MoEConfig("s1k8", T=97, d=384, E=32, k=8, S=1, I=256, bias="normal0.05"),
      None),
@@ -121,7 +121,7 @@ def test_backward_full_size_slice(T):
     the paired-CTA GEMMs of prefill-sized batches): dx, dWg and the shared
     experts' gradients in full, the routed experts' gradients on a seeded
     sample of experts."""
-    cfg = CONFIGS[4]
+    cfg = FWD_BWD
     inp = make_inputs(cfg, T=T, device="cuda")
     y_inf, y, grads, idx = _run(inp)
     rng = np.random.default_rng(4)

@@ -16,7 +16,7 @@ import pytest
 import torch
 
 from fine_grained_moe_fp32_b200 import moe as M
-from fine_grained_moe_fp32_b200.workloads import CONFIGS, MoEConfig, make_inputs, small_config
+from fine_grained_moe_fp32_b200.workloads import (MoEConfig, make_inputs, small_config, FWD_BWD, PREFILL_SKEWED, TINY)
 from oracle import moe_oracle as O
 import parity_utils as PU
 
@@ -82,9 +82,9 @@ def _check_bias(inp, layer, v, gamma=GAMMA, train=False):
 
 
 SMALL = [
-    ("tiny_L64", CONFIGS[0], None, 64),
-    ("tiny_L1", CONFIGS[0], None, 1),
-    ("tiny_L256_one_seq", CONFIGS[0], None, 256),
+    ("tiny_L64", TINY, None, 64),
+    ("tiny_L1", TINY, None, 1),
+    ("tiny_L256_one_seq", TINY, None, 256),
     ("E16_T300_L100_ragged_chunks", small_config(T=300, d=256, E=16, k=4, I=128), None, 100),
     ("E8_k1_T77_L7", MoEConfig("e8k1", T=77, d=128, E=8, k=1, S=1, I=64, bias="uniform0.01"),
      None, 7),
@@ -108,7 +108,7 @@ def test_balance_small(name, cfg, T, seq_len):
 def test_balance_full_size_skewed_prefill():
     """T=16384 skewed routing (most pairs on a few experts, many experts
     empty) in 4 sequences of 4096 tokens."""
-    inp, layer, v = _routed(CONFIGS[3])
+    inp, layer, v = _routed(PREFILL_SKEWED)
     st, ref = _check_stats(inp, layer, v, 4096)
     assert (st["f"].cpu().numpy() == 0).any()          # empty experts inside a sequence
     _check_bias(inp, layer, v)
@@ -117,7 +117,7 @@ def test_balance_full_size_skewed_prefill():
 def test_balance_full_size_fwd_bwd_workload():
     """The fwd+bwd workload (T=8192, one 8192-token sequence) after
     moe_forward_train, reading the training workspace."""
-    inp, layer, v = _routed(CONFIGS[4], train=True)
+    inp, layer, v = _routed(FWD_BWD, train=True)
     _check_stats(inp, layer, v, 8192, train=True)
     _check_bias(inp, layer, v, train=True)
 
@@ -164,7 +164,7 @@ def test_balance_bad_ids_flagged_and_skipped():
 
 
 def test_bias_update_in_place_and_determinism():
-    inp, layer, v = _routed(CONFIGS[0])
+    inp, layer, v = _routed(TINY)
     T = inp["T"]
     a = layer.balance_stats(T, 64, ALPHA, train=False)
     b = layer.balance_stats(T, 64, ALPHA, train=False)

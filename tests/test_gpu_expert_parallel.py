@@ -15,7 +15,7 @@ import pytest
 import torch
 
 from fine_grained_moe_fp32_b200 import moe as M
-from fine_grained_moe_fp32_b200.workloads import CONFIGS, MoEConfig, make_inputs, small_config
+from fine_grained_moe_fp32_b200.workloads import (CONFIGS, MoEConfig, make_inputs, small_config, DECODE, TINY)
 from oracle import moe_oracle as O
 import parity_utils as PU
 
@@ -88,7 +88,7 @@ def _check_outputs(inp, xs, ys, ep, spec):
 def test_ep_one_rank_is_moe_forward_bit_for_bit():
     """One rank: the receive buffer is the permutation's x_perm and the layer
     output is moe_forward's, bit for bit."""
-    inp, xs = _ranks(CONFIGS[0], 1)
+    inp, xs = _ranks(TINY, 1)
     ep, ys, st = _run(inp, xs, 1)
     assert st == M.MOE_OK
     layer = M.MoELayer(inp)
@@ -102,10 +102,10 @@ def test_ep_one_rank_is_moe_forward_bit_for_bit():
 
 
 EP_CASES = [
-    ("tiny_W2", CONFIGS[0], 2, None, 16),
-    ("tiny_W4", CONFIGS[0], 4, None, 16),
-    ("tiny_W8", CONFIGS[0], 8, None, 16),
-    ("tiny_W4_align128", CONFIGS[0], 4, None, 128),
+    ("tiny_W2", TINY, 2, None, 16),
+    ("tiny_W4", TINY, 4, None, 16),
+    ("tiny_W8", TINY, 8, None, 16),
+    ("tiny_W4_align128", TINY, 4, None, 128),
     ("E16_T77_W4_ragged", small_config(T=77, d=256, E=16, k=4, I=128), 4, None, 16),
     ("E16_T40_W16_one_expert_per_rank", small_config(T=40, d=256, E=16, k=4, I=128), 16,
      None, 16),
@@ -171,7 +171,7 @@ def test_ep_rejected_count_table_sends_nothing():
 
 
 def test_ep_deterministic():
-    inp, xs = _ranks(CONFIGS[0], 4)
+    inp, xs = _ranks(TINY, 4)
     ep = M.EPRanks(inp, 4, xs[0].shape[0])
     a = [y.clone() for y in ep(xs)]
     b = ep(xs)
@@ -185,7 +185,7 @@ def test_ep_full_size_decode_8_ranks():
     emulated ranks of 16 experts: every rank's layout and dispatched rows bit
     for bit, the output on a seeded sample of every rank's tokens against the
     per-token oracle, and against the single-GPU layer on the same tokens."""
-    cfg = CONFIGS[1]
+    cfg = DECODE
     W = 8
     inp, xs = _ranks(cfg, W)
     ep, ys, st = _run(inp, xs, W)

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from fine_grained_moe_fp32_b200 import moe as M
-from fine_grained_moe_fp32_b200.workloads import CONFIGS, MoEConfig, make_inputs, small_config
+from fine_grained_moe_fp32_b200.workloads import (CONFIGS, MoEConfig, make_inputs, small_config, DECODE, PREFILL_BALANCED, PREFILL_SKEWED, TINY)
 from oracle import moe_oracle as O
 import parity_utils as PU
 
@@ -67,15 +67,15 @@ def _check_permutation(dm, pm, idx_gpu, x):
 # ------------------------------------------------------------------ router
 
 ROUTE_CASES = [
-    ("tiny_full", CONFIGS[0], None),
+    ("tiny_full", TINY, None),
     ("small_E16_ragged", small_config(T=300, d=256, E=16, k=4, I=128), None),
     ("E8_k1", MoEConfig("e8k1", T=77, d=128, E=8, k=1, S=1, I=64, bias="uniform0.01"), None),
     ("E128_k8", MoEConfig("k8", T=129, d=384, E=128, k=8, S=2, I=64, bias="normal0.05"), None),
-    ("decode_full", CONFIGS[1], None),
+    ("decode_full", DECODE, None),
     # 46 and 18 split partials: the top-k sums them with 4 and 2 warps per token
-    ("d5120_T300_46_splits", CONFIGS[1], 300),
-    ("d5120_T1024_18_splits", CONFIGS[2], 1024),
-    ("skewed_zipf_slice", CONFIGS[3], 2048),
+    ("d5120_T300_46_splits", DECODE, 300),
+    ("d5120_T1024_18_splits", PREFILL_BALANCED, 1024),
+    ("skewed_zipf_slice", PREFILL_SKEWED, 2048),
 ]
 
 
@@ -159,10 +159,10 @@ def test_permute_flags_bad_expert_ids():
 # ------------------------------------------------------------------ grouped GEMMs
 
 GEMM_CASES = [
-    ("tiny_full", CONFIGS[0], None, 16),
-    ("tiny_align128", CONFIGS[0], None, 128),
+    ("tiny_full", TINY, None, 16),
+    ("tiny_align128", TINY, None, 128),
     ("small_ragged", small_config(T=333, d=256, E=16, k=4, I=192), None, 16),
-    ("decode_full", CONFIGS[1], None, 16),
+    ("decode_full", DECODE, None, 16),
     ("pair_prefill_T700", small_config(T=700, d=512, E=16, k=4, I=256), None, 16),
 ]
 
@@ -235,8 +235,8 @@ def _forward(inp, align=16):
 
 
 FWD_CASES = [
-    ("tiny_full", CONFIGS[0], None, 16),
-    ("tiny_align128", CONFIGS[0], None, 128),
+    ("tiny_full", TINY, None, 16),
+    ("tiny_align128", TINY, None, 128),
     ("small_ragged_T333", small_config(T=333, d=256, E=16, k=4, I=192), None, 16),
     ("single_token", small_config(T=1, d=256, E=16, k=4, I=128), None, 16),
     ("pair_prefill_T700", small_config(T=700, d=512, E=16, k=4, I=256), None, 16),
@@ -290,11 +290,12 @@ def test_forward_deterministic():
 
 # ------------------------------------------------------------------ full-size configurations
 
-@pytest.mark.parametrize("cid,n_sample", [(1, 24), (2, 12), (3, 12)])
-def test_forward_full_size_sampled(cid, n_sample):
+@pytest.mark.parametrize("cfg,n_sample,seed",
+                         [(DECODE, 24, 1), (PREFILL_BALANCED, 12, 2), (PREFILL_SKEWED, 12, 3)],
+                         ids=["decode", "prefill_balanced", "prefill_skewed"])
+def test_forward_full_size_sampled(cfg, n_sample, seed):
     """The full configuration on the device: the whole routing and permutation
     are compared; the output on a seeded sample of tokens (per-token oracle)."""
-    cfg = CONFIGS[cid]
     inp = make_inputs(cfg, device=DEV)
     layer = M.MoELayer(inp)
     y = layer(inp["x"])
@@ -310,7 +311,7 @@ def test_forward_full_size_sampled(cid, n_sample):
     np.testing.assert_array_equal(v["offsets"].cpu().numpy(), pm["offsets"])
     np.testing.assert_array_equal(v["row_of"].cpu().numpy(), pm["row_of"])
     np.testing.assert_array_equal(v["token_of_row"].cpu().numpy(), pm["token_of_row"])
-    rng = np.random.default_rng(cid)
+    rng = np.random.default_rng(seed)
     toks = np.sort(rng.choice(cfg.T, size=n_sample, replace=False))
     ref = O.forward_tokens(host, toks, idx=idx_gpu[toks])
     PU.check_output(y[torch.as_tensor(toks, device=DEV)], ref["y"], "y (sampled)")

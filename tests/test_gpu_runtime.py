@@ -53,16 +53,17 @@ def test_phase_events_cover_the_step():
     assert sum(parts) <= outer[0].elapsed_time(outer[1]) * 1.01 + 0.05
 
 
-@pytest.mark.parametrize("cid,T", [(0, None), (1, None), (2, 1024)],
+@pytest.mark.parametrize("name,T", [("TINY", None), ("DECODE", None), ("PREFILL_BALANCED", 1024)],
                          ids=["tiny", "decode", "prefill_T1024_cta_pairs"])
-def test_forward_captures_into_a_cuda_graph(cid, T):
+def test_forward_captures_into_a_cuda_graph(name, T):
     """moe_forward issues only stream work (no host sync, no allocation), so it
     can be captured once and replayed: every replay gives the eager result bit
     for bit, and a replay follows new input values written in place."""
     import torch
     from fine_grained_moe_fp32_b200 import moe as M
-    from fine_grained_moe_fp32_b200.workloads import CONFIGS, make_inputs
-    cfg = CONFIGS[cid]
+    from fine_grained_moe_fp32_b200 import workloads as W
+    cfg = getattr(W, name)
+    make_inputs = W.make_inputs
     inp = make_inputs(cfg, device="cuda", T=T)
     layer = M.MoELayer(inp)
     x = inp["x"].clone()

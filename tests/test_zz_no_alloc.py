@@ -9,7 +9,7 @@ import pytest
 import torch
 
 from fine_grained_moe_fp32_b200 import moe as M
-from fine_grained_moe_fp32_b200.workloads import CONFIGS, make_inputs
+from fine_grained_moe_fp32_b200.workloads import make_inputs, PREFILL_BALANCED, TINY
 
 pytestmark = pytest.mark.gpu
 
@@ -34,7 +34,7 @@ def _no_alloc(dm, g):
 
 
 def test_no_alloc_route_matches_moe_route_on_two_calls():
-    cases = [(CONFIGS[2], 4096, 0), (CONFIGS[0], 256, 3)]   # big call first, then a small one
+    cases = [(PREFILL_BALANCED, 4096, 0), (TINY, 256, 3)]   # big call first, then a small one
     for cfg, T, seed in cases:
         inp = make_inputs(cfg, T=T, seed=seed, weights=False)
         g = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
