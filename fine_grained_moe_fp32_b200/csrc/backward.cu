@@ -19,8 +19,8 @@ namespace {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
-         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+  const __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);  // one paired cvt, lo in the low half
+  return *reinterpret_cast<const uint32_t*>(&h2);
 }
 
 constexpr int kCbThreads = 128;

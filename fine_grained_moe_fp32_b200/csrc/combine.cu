@@ -90,9 +90,8 @@ combine_kernel(Rows src, const float* __restrict__ topk_w, const float* __restri
     uint32_t o[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * i]));
-      const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * i + 1]));
-      o[i] = lo | (hi << 16);
+      const __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+      o[i] = *reinterpret_cast<const uint32_t*>(&h2);
     }
     reinterpret_cast<uint4*>(y + (size_t)t * d)[v] = make_uint4(o[0], o[1], o[2], o[3]);
   }

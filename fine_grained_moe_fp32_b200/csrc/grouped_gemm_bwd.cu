@@ -448,8 +448,8 @@ grouped_gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmA_r,
               for (int i = 0; i < 4; ++i) {
                 const float lo = zero ? 0.f : __uint_as_float(v[j8 * 8 + 2 * i]);
                 const float hi = zero ? 0.f : __uint_as_float(v[j8 * 8 + 2 * i + 1]);
-                w[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
-                       ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);  // one paired cvt
+                w[i] = *reinterpret_cast<const uint32_t*>(&h2);
               }
               *reinterpret_cast<uint4*>(dst + j8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
             }

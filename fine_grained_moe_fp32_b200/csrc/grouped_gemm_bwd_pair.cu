@@ -38,19 +38,21 @@ namespace {
 
 enum PBwdMode : int { kPDgradDown = 0, kPDgradUp = 1, kPWgrad = 2 };
 
-constexpr int kBK = 128;            // K per stage: two 64-deep sub-blocks
+constexpr int kBK = 128;            // dgrads: K per stage, two 64-deep sub-blocks
 constexpr int kSubK = 64;
 constexpr int kMnBlk = 8192;        // one MN-major box: 64 MN x 64 K rows of bf16
 constexpr int kASub = 2 * kMnBlk;   // this CTA's 128 A rows for one K sub-block
-constexpr int kABytes = 2 * kASub;
+
 constexpr int kBoxB = 128;          // token rows per K-major B box (this CTA's half)
 constexpr int kBSub = 128 * 128;    // one K sub-block of this CTA's B (either layout)
-constexpr int kBBytes = 2 * kBSub;
-constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kStages = 3;
+constexpr int kMaxStages = 6;
+// weight gradients: stage depth and count (the same 192 KB in flight as 6
+// stages of 64 measured 3-5 % slower than 3 stages of 128)
+constexpr int kWgradKSubs = 2, kWgradStages = 3;
 constexpr int kNT = 256;            // N per pair tile
 constexpr int kThreads = 224;       // warp 0 A producer, 1 MMA, 2-5 epilogue, 6 B producer
 constexpr int kEpiThreads = 128;
+constexpr int kEpiWarps = kEpiThreads / 32;
 constexpr uint32_t kTmemCols = 2 * kNT;
 constexpr int kMaxGroups = 136;     // 128 routed + up to 8 shared groups
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
@@ -93,8 +95,8 @@ struct PBTile {
 };
 
 struct PBCtl {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -130,7 +132,7 @@ __device__ __forceinline__ uint32_t idesc_pbwd(uint32_t n, bool b_mn) {
          ((n >> 3) << 17) | ((256u >> 4) << 24);
 }
 
-template <int MODE>
+template <int MODE, int BK>
 __device__ __forceinline__ PBTile pb_decode(const PBCtl& c, const PBParams& p, int tile) {
   int lo = 0, hi = c.ngroups - 1;
   while (lo < hi) {
@@ -150,8 +152,8 @@ __device__ __forceinline__ PBTile pb_decode(const PBCtl& c, const PBParams& p, i
     t.n = min(kNT, ntot - t.ncol0);
     t.row0 = c.row0[lo];
     t.nrows = c.rows[lo];
-    t.kchunks = (t.nrows + kBK - 1) / kBK;
-    const int rem = t.nrows - (t.kchunks - 1) * kBK;
+    t.kchunks = (t.nrows + BK - 1) / BK;
+    const int rem = t.nrows - (t.kchunks - 1) * BK;
     t.last_k16 = t.kchunks > 0 ? (rem + 15) / 16 : 0;
   } else {
     const int mtn = routed ? p.mt_routed : p.mt_shared;
@@ -162,14 +164,15 @@ __device__ __forceinline__ PBTile pb_decode(const PBCtl& c, const PBParams& p, i
     t.n = (t.nrows + 15) & ~15;
     t.ncol0 = 0;
     t.kchunks = routed ? p.kit_routed : p.kit_shared;
-    t.last_k16 = kBK / 16;
+    t.last_k16 = BK / 16;
   }
   return t;
 }
 
 __device__ __forceinline__ float pb_sigmoid(float g) { return 1.0f / (1.0f + __expf(-g)); }
 
-template <int MODE>
+// KSUBS 64-deep K sub-blocks per stage, STAGES stages in the ring.
+template <int MODE, int KSUBS, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
                              const __grid_constant__ CUtensorMap tmA2_r,
@@ -181,6 +184,10 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
                              const __grid_constant__ CUtensorMap tmO2_r,
                              const __grid_constant__ CUtensorMap tmO_s,
                              const __grid_constant__ CUtensorMap tmO2_s, const PBParams p) {
+  constexpr int BK = KSUBS * kSubK;
+  constexpr int kABytes = KSUBS * kASub;
+  constexpr int kStageBytes = kABytes + KSUBS * kBSub;
+  static_assert(STAGES <= kMaxStages, "barrier arrays");
   __shared__ PBCtl ctl;
   extern __shared__ uint8_t dsmem_raw[];
   const uint32_t raw = smem_u32(dsmem_raw);
@@ -188,7 +195,7 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
   // epilogue staging, 32 KB: the SwiGLU backward's g then u tiles ([32][128]
   // bf16 each), or per epilogue warp two 4 KB store buffers of the weight
   // gradients (32 rows x 64 columns of bf16, 128-byte swizzle)
-  uint8_t* epi = dsmem_raw + (sbase - raw) + kStages * kStageBytes;
+  uint8_t* epi = dsmem_raw + (sbase - raw) + STAGES * kStageBytes;
   uint16_t* epi_g = reinterpret_cast<uint16_t*>(epi);
   uint16_t* epi_u = epi_g + 32 * 128;
 
@@ -245,13 +252,13 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
       ctl.ngroups = G;
     }
     if (lane == 0) {
-      for (int s = 0; s < kStages; ++s) {
+      for (int s = 0; s < STAGES; ++s) {
         mbar_init(smem_u32(&ctl.full[s]), 2);  // armed by both of the leader's producers
         mbar_init(smem_u32(&ctl.empty[s]), 1);
       }
       for (int b = 0; b < 2; ++b) {
         mbar_init(smem_u32(&ctl.tfull[b]), 1);
-        mbar_init(smem_u32(&ctl.tempty[b]), 2 * kEpiThreads);  // both CTAs' epilogues
+        mbar_init(smem_u32(&ctl.tempty[b]), 2 * kEpiWarps);  // one lane per epilogue warp, both CTAs
       }
       mbar_init(smem_u32(&ctl.drain), 1);
       ctl.abort_flag = 0;
@@ -285,7 +292,7 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
       uint32_t armed = 0, armed_parity = 0;  // leader: stages whose full phase it armed
       bool ok = true;
       for (int tile = pair; tile < total && ok; tile += npairs) {
-        const PBTile t = pb_decode<MODE>(ctl, p, tile);
+        const PBTile t = pb_decode<MODE, BK>(ctl, p, tile);
         const bool routed = t.g < p.E;
         const int s_idx = t.g - p.E;
         const int r0 = t.mt * 256 + (int)rank * 128;  // this CTA's first M row
@@ -294,9 +301,9 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
         if (wA) {
           tx_pair = 2u * kABytes;
         } else if (MODE == kPWgrad) {
-          tx_pair = 2u * 2u * (uint32_t)((half / 64) * kMnBlk);
+          tx_pair = 2u * KSUBS * (uint32_t)((half / 64) * kMnBlk);
         } else {
-          tx_pair = 2u * 2u * (uint32_t)(kBoxB * 128);
+          tx_pair = 2u * KSUBS * (uint32_t)(kBoxB * 128);
         }
         // A coordinates that do not change along K
         int a_x = 0, a_plane = 0;
@@ -338,8 +345,8 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
           }
           const uint32_t sA = sbase + stage * kStageBytes;
           const uint32_t sB = sA + kABytes;
-          for (int j = 0; j < 2; ++j) {  // the two 64-deep K sub-blocks
-            const int kj = kc * kBK + j * kSubK;
+          for (int j = 0; j < KSUBS; ++j) {  // the 64-deep K sub-blocks
+            const int kj = kc * BK + j * kSubK;
             if (wA) {
               if (MODE == kPDgradDown) {
                 // A = W2^T: K rows d of W2 [.., d, I], M columns = features
@@ -353,7 +360,7 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
                 const bool second = kc >= ks;
                 const CUtensorMap* tAk =
                     routed ? (second ? &tmA2_r : &tmA_r) : (second ? &tmA2_s : &tmA_s);
-                const int krow = (second ? kj - ks * kBK : kj) + (routed ? t.g * p.I : 0);
+                const int krow = (second ? kj - ks * BK : kj) + (routed ? t.g * p.I : 0);
                 for (int h = 0; h < 2; ++h)
                   tma_load_3d_pair(sA + j * kASub + h * kMnBlk, tAk, fb, a_x + h * 64, krow, 0,
                                    pol);
@@ -373,12 +380,12 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
               }
             }
           }
-          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
       if (leader) {
         // every phase this CTA armed completes only once both CTAs' bytes land
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < STAGES; ++s) {
           if (((armed >> s) & 1u) &&
               !mbar_wait_bounded(smem_u32(&ctl.full[s]), (armed_parity >> s) & 1u, kDrainLimitNs))
             pb_timeout(ctl, p);
@@ -400,7 +407,7 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = pair; tile < total && ok; tile += npairs) {
-        const PBTile t = pb_decode<MODE>(ctl, p, tile);
+        const PBTile t = pb_decode<MODE, BK>(ctl, p, tile);
         const uint32_t idesc = idesc_pbwd((uint32_t)t.n, MODE == kPWgrad);
         if (pb_aborted(ctl) ||
             !mbar_wait_bounded(smem_u32(&ctl.tempty[acc]), acc_phase ^ 1u, p.wait_limit_ns)) {
@@ -419,7 +426,7 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
           tc_fence_after();
           const uint32_t sA = sbase + stage * kStageBytes;
           const uint32_t sB = sA + kABytes;
-          const int nk16 = (kc == t.kchunks - 1) ? t.last_k16 : kBK / 16;
+          const int nk16 = (kc == t.kchunks - 1) ? t.last_k16 : BK / 16;
           for (int k8 = 0; k8 < nk16; ++k8) {
             const uint32_t offa = (k8 >> 2) * kASub + (k8 & 3) * 2048;
             const uint64_t ad = sdesc_mn_sw128(sA + offa);
@@ -429,7 +436,7 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
             mma_bf16_ss_pair(dt, ad, bd, idesc, (kc | k8) != 0 ? 1u : 0u);
           }
           mma_commit_pair(smem_u32(&ctl.empty[stage]), 0x3);
-          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         mma_commit_pair(smem_u32(&ctl.tfull[acc]), 0x3);
@@ -470,8 +477,21 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t nstore = 0;  // weight-gradient chunks this CTA has handed to TMA
+    // hand the accumulator back to the MMA warp: every lane's TMEM reads have
+    // completed (tcgen05.wait::ld), then one lane per warp arrives on the
+    // leader's barrier (one arrival instead of 32 remote ones)
+    auto release = [&](int a) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(smem_u32(&ctl.tempty[a]));
+        else
+          mbar_arrive_remote(a ? tempty_leader1 : tempty_leader0);
+      }
+    };
     for (int tile = pair; tile < total; tile += npairs) {
-      const PBTile t = pb_decode<MODE>(ctl, p, tile);
+      const PBTile t = pb_decode<MODE, BK>(ctl, p, tile);
       const bool routed = t.g < p.E;
       const int r0 = t.mt * 256 + (int)rank * 128;
       // rows past the group's M extent hold zero-filled products: skipped
@@ -486,6 +506,7 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
       tc_fence_after();
       const uint32_t tbase = tmem_base + (uint32_t)(acc * kNT) + ((uint32_t)(q * 32) << 16);
       const int ncols = MODE == kPWgrad ? t.n : t.nrows;
+      bool freed = false;
       if (MODE == kPWgrad && live) {
         // dW[group][row0 + mrow][ncol0 + c0 .. + 64] in bf16.  Each warp owns
         // 32 rows: it stages its 32 x 64 block (128-byte rows, 128-byte
@@ -503,8 +524,8 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
           for (int i = 0; i < 16; ++i) {
             const float lo = zero ? 0.f : __uint_as_float(v[2 * i]);
             const float hi = zero ? 0.f : __uint_as_float(v[2 * i + 1]);
-            w[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
-                   ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);  // one paired cvt
+            w[i] = *reinterpret_cast<const uint32_t*>(&h2);
           }
         };
         // tile widths are multiples of 64: columns go 64 at a time (va, vb)
@@ -512,6 +533,10 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
         tmem_ld_32x32b_x32(tbase, va);
         tmem_ld_32x32b_x32(tbase + 32u, vb);
         tmem_ld_wait();
+        if (ncols <= 64) {  // every column is in registers: the MMAs may go on
+          release(acc);
+          freed = true;
+        }
         for (int c0 = 0; c0 < ncols; c0 += 64) {
           uint32_t wa[16], wb[16];
           pack(va, wa);
@@ -538,7 +563,13 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
             bulk_commit_group();
           }
           ++nstore;
-          if (more) tmem_ld_wait();
+          if (more) {
+            tmem_ld_wait();
+            if (c0 + 128 >= ncols) {  // those were the last columns
+              release(acc);
+              freed = true;
+            }
+          }
         }
       }
       for (int c0 = 0; MODE != kPWgrad && live && c0 < ncols; c0 += 32) {
@@ -595,11 +626,7 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
             if (j < nj) out[(size_t)(t.row0 + c0 + j) * ldo + col] = __uint_as_float(v[j]);
         }
       }
-      tc_fence_before();
-      if (leader)
-        mbar_arrive(smem_u32(&ctl.tempty[acc]));
-      else
-        mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
+      if (!freed) release(acc);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
     if (MODE == kPWgrad && lane == 0) bulk_wait_group<0>();  // every store has landed
@@ -659,11 +686,11 @@ bool make_store_map3(CUtensorMap* m, void* base, uint64_t inner, uint64_t rows, 
 }
 
 // m[0..5]: operand maps; m[6..9]: output maps of the weight gradients.
-template <int MODE>
+template <int MODE, int KSUBS, int STAGES>
 cudaError_t launch_pb(const CUtensorMap* m, const PBParams& p, int num_sms, cudaStream_t st) {
-  constexpr size_t smem = (size_t)kStages * kStageBytes + 32768 + 1024;
+  constexpr size_t smem = (size_t)STAGES * KSUBS * (kASub + kBSub) + 32768 + 1024;
   static_assert(smem + sizeof(PBCtl) <= 232448, "shared memory budget");
-  auto kern = grouped_gemm_bwd_pair_kernel<MODE>;
+  auto kern = grouped_gemm_bwd_pair_kernel<MODE, KSUBS, STAGES>;
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
@@ -753,7 +780,7 @@ cudaError_t launch_backward_gemms_pair(const Shape& s, const BackwardGemmArgs& a
     p.ld_gu_shared = SI;
     p.ucol_routed = s.I;
     p.ucol_shared = SI;
-    if ((err = launch_pb<kPDgradDown>(m, p, num_sms, st)) != cudaSuccess) return err;
+    if ((err = launch_pb<kPDgradDown, 2, 3>(m, p, num_sms, st)) != cudaSuccess) return err;
     if ((err = mark(0)) != cudaSuccess) return err;
   }
   // ---- dW2 = dY^T H (routed) and dWs2[s] = dy^T H_shared[:, s]
@@ -780,7 +807,7 @@ cudaError_t launch_backward_gemms_pair(const Shape& s, const BackwardGemmArgs& a
     p.ntot_routed = p.ntot_shared = s.I;
     p.nt_routed = p.nt_shared = (int)ceil_div(s.I, kNT);
     p.b_step_shared = s.I;
-    if ((err = launch_pb<kPWgrad>(m, p, num_sms, st)) != cudaSuccess) return err;
+    if ((err = launch_pb<kPWgrad, kWgradKSubs, kWgradStages>(m, p, num_sms, st)) != cudaSuccess) return err;
     if ((err = mark(1)) != cudaSuccess) return err;
   }
   // ---- dX = dG W1 + dU W3 (token rows), fp32
@@ -808,7 +835,7 @@ cudaError_t launch_backward_gemms_pair(const Shape& s, const BackwardGemmArgs& a
     p.ld_routed = s.d;
     p.out_shared = a.dx_shared;
     p.ld_shared = s.d;
-    if ((err = launch_pb<kPDgradUp>(m, p, num_sms, st)) != cudaSuccess) return err;
+    if ((err = launch_pb<kPDgradUp, 2, 3>(m, p, num_sms, st)) != cudaSuccess) return err;
     if ((err = mark(2)) != cudaSuccess) return err;
   }
   // ---- [dW1 ; dW3] = [dG | dU]^T X in one launch (routed: x_perm; shared: x)
@@ -842,7 +869,7 @@ cudaError_t launch_backward_gemms_pair(const Shape& s, const BackwardGemmArgs& a
     p.a_step_shared = s.I;
     p.ntot_routed = p.ntot_shared = s.d;
     p.nt_routed = p.nt_shared = (int)ceil_div(s.d, kNT);
-    if ((err = launch_pb<kPWgrad>(m, p, num_sms, st)) != cudaSuccess) return err;
+    if ((err = launch_pb<kPWgrad, kWgradKSubs, kWgradStages>(m, p, num_sms, st)) != cudaSuccess) return err;
   }
   return mark(3);
 }

@@ -196,7 +196,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
       }
       for (int b = 0; b < 2; ++b) {
         mbar_init(smem_u32(&ctl.tfull[b]), 1);
-        mbar_init(smem_u32(&ctl.tempty[b]), 2 * kEpiThreads);  // both CTAs' epilogues
+        mbar_init(smem_u32(&ctl.tempty[b]), 2 * (kEpiThreads / 32));  // a lane per epilogue warp
       }
       mbar_init(smem_u32(&ctl.drain), 1);
       ctl.abort_flag = 0;
@@ -422,11 +422,16 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
           named_bar_sync(1, kEpiThreads);
         }
       }
+      // every lane's TMEM reads are done: one lane per warp hands the
+      // accumulator back (one arrival instead of 32 remote ones)
       tc_fence_before();
-      if (leader)
-        mbar_arrive(smem_u32(&ctl.tempty[acc]));
-      else
-        mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(smem_u32(&ctl.tempty[acc]));
+        else
+          mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
+      }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
   }
