@@ -50,9 +50,16 @@ constexpr int kMaxStages = 6;
 // stages of 64 measured 3-5 % slower than 3 stages of 128)
 constexpr int kWgradKSubs = 2, kWgradStages = 3;
 constexpr int kNT = 256;            // N per pair tile
-constexpr int kThreads = 224;       // warp 0 A producer, 1 MMA, 2-5 epilogue, 6 B producer
-constexpr int kEpiThreads = 128;
-constexpr int kEpiWarps = kEpiThreads / 32;
+// Warp 0 A producer, 1 MMA, 2 .. 1 + epi_warps(MODE) epilogue, the next one
+// B producer.  The weight gradients and the dH dgrad run 8 epilogue warps
+// (two per TMEM lane quarter): the weight gradients' tiles are short (K = one
+// segment's few hundred tokens) and the dH epilogue carries the SwiGLU
+// backward, so with 4 warps their epilogues would pace the MMAs.  The
+// weight-gradient warps take alternate 64-column blocks, the dH warps form two
+// groups of 4 that take alternate 32-token chunks.
+constexpr int epi_warps(int mode) { return mode == 1 ? 4 : 8; }
+constexpr int block_threads(int mode) { return 32 * (3 + epi_warps(mode)); }
+constexpr int kEpiStaging = 32768;  // epilogue staging bytes, shared by the epilogue warps
 constexpr uint32_t kTmemCols = 2 * kNT;
 constexpr int kMaxGroups = 136;     // 128 routed + up to 8 shared groups
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
@@ -173,7 +180,7 @@ __device__ __forceinline__ float pb_sigmoid(float g) { return 1.0f / (1.0f + __e
 
 // KSUBS 64-deep K sub-blocks per stage, STAGES stages in the ring.
 template <int MODE, int KSUBS, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(block_threads(MODE), 1)
 grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
                              const __grid_constant__ CUtensorMap tmA2_r,
                              const __grid_constant__ CUtensorMap tmB_r,
@@ -184,6 +191,15 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
                              const __grid_constant__ CUtensorMap tmO2_r,
                              const __grid_constant__ CUtensorMap tmO_s,
                              const __grid_constant__ CUtensorMap tmO2_s, const PBParams p) {
+  static_assert(epi_warps(kPDgradUp) == 4 && epi_warps(kPWgrad) == 8 &&
+                    epi_warps(kPDgradDown) == 8,
+                "epi_warps keys on the mode values");
+  constexpr int kEpiWarps = epi_warps(MODE);
+  constexpr int kEpiThreads = 32 * kEpiWarps;
+  constexpr int kBWarp = 2 + kEpiWarps;  // B producer
+  // weight-gradient store buffers per epilogue warp (4 KB each: 32 rows x 64 columns)
+  constexpr int kBufs = kEpiStaging / 4096 / kEpiWarps;
+  static_assert(kBufs >= 1, "staging");
   constexpr int BK = KSUBS * kSubK;
   constexpr int kABytes = KSUBS * kASub;
   constexpr int kStageBytes = kABytes + KSUBS * kBSub;
@@ -192,12 +208,11 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
   extern __shared__ uint8_t dsmem_raw[];
   const uint32_t raw = smem_u32(dsmem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
-  // epilogue staging, 32 KB: the SwiGLU backward's g then u tiles ([32][128]
-  // bf16 each), or per epilogue warp two 4 KB store buffers of the weight
-  // gradients (32 rows x 64 columns of bf16, 128-byte swizzle)
+  // epilogue staging, 32 KB: per dH epilogue group the SwiGLU backward's g
+  // then u tiles ([32][128] bf16 each), or per weight-gradient epilogue warp
+  // one 4 KB store buffer (32 rows x 64 columns of bf16, 128-byte swizzle)
   uint8_t* epi = dsmem_raw + (sbase - raw) + STAGES * kStageBytes;
   uint16_t* epi_g = reinterpret_cast<uint16_t*>(epi);
-  uint16_t* epi_u = epi_g + 32 * 128;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -280,7 +295,7 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
   const int pair = (int)cluster_id_x();
   const int npairs = (int)nclusters_x();
 
-  if (warp == 0 || warp == 6) {
+  if (warp == 0 || warp == kBWarp) {
     // ========== TMA producers (both CTAs): warp 0 operand A, warp 6 operand B ==========
     if (lane == 0) {
       const bool wA = warp == 0;
@@ -446,10 +461,21 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
       if (!mbar_wait_bounded(smem_u32(&ctl.drain), 0, kDrainLimitNs)) pb_timeout(ctl, p);
     }
   } else {
-    // ================= epilogue (warps 2..5, both CTAs) =================
-    const int q = warp & 3;
+    // ============ epilogue (warps 2 .. kBWarp - 1, both CTAs) ============
+    const int q = warp & 3;          // TMEM lane quarter a warp may read
     const int mrow = q * 32 + lane;  // accumulator row = TMEM lane
-    const int et = threadIdx.x - 64; // 0..127 over the epilogue warps
+    const int et = threadIdx.x - 64; // 0 .. kEpiThreads - 1 over the epilogue warps
+    const int ew = warp - 2;         // epilogue warp index
+    // dH dgrad: two groups of 4 warps, each over all 128 TMEM lanes, take
+    // alternate 32-token chunks with their own staging and named barrier
+    constexpr bool kGroups = MODE == kPDgradDown && kEpiWarps == 8;
+    constexpr int kGrpThreads = 128;
+    constexpr int kChunkStep = kGroups ? 64 : 32;
+    const int grp = kGroups ? (ew >> 2) : 0;
+    const int eg = et & (kGrpThreads - 1);  // thread index inside the group
+    uint16_t* const gbuf = epi_g + grp * (2 * 32 * 128);
+    uint16_t* const ubuf = gbuf + 32 * 128;
+    const int gbar = 1 + 2 * grp;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&ctl.tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&ctl.tempty[1]), 0);
     // SwiGLU backward: this thread's share of the g / u rows of one 32-token
@@ -463,7 +489,7 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
       const int nj = min(32, t.nrows - c0);
 #pragma unroll
       for (int it = 0; it < 4; ++it) {
-        const int i = et + it * kEpiThreads;
+        const int i = eg + it * kGrpThreads;
         const int r = i >> 4, cv = i & 15;
         gpre[it] = make_uint4(0, 0, 0, 0);
         upre[it] = gpre[it];
@@ -496,7 +522,7 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
       const int r0 = t.mt * 256 + (int)rank * 128;
       // rows past the group's M extent hold zero-filled products: skipped
       const bool live = r0 < (routed ? p.mext_routed : p.mext_shared);
-      if (MODE == kPDgradDown && live) load_gu(t, r0, 0);
+      if (MODE == kPDgradDown && live) load_gu(t, r0, grp * 32);
       bool bad = pb_aborted(ctl);
       if (!bad && !mbar_wait_bounded(smem_u32(&ctl.tfull[acc]), acc_phase, p.wait_limit_ns)) {
         pb_timeout(ctl, p);
@@ -528,26 +554,32 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
             w[i] = *reinterpret_cast<const uint32_t*>(&h2);
           }
         };
-        // tile widths are multiples of 64: columns go 64 at a time (va, vb)
+        // tile widths are multiples of 64: columns go 64 at a time (va, vb);
+        // the warps sharing a lane quarter take alternate 64-column blocks
+        constexpr int kStep = 64 * (kEpiWarps / 4);
+        const int cfirst = 64 * (ew >> 2);
         uint32_t va[32], vb[32];
-        tmem_ld_32x32b_x32(tbase, va);
-        tmem_ld_32x32b_x32(tbase + 32u, vb);
-        tmem_ld_wait();
-        if (ncols <= 64) {  // every column is in registers: the MMAs may go on
+        if (cfirst < ncols) {
+          tmem_ld_32x32b_x32(tbase + (uint32_t)cfirst, va);
+          tmem_ld_32x32b_x32(tbase + (uint32_t)(cfirst + 32), vb);
+          tmem_ld_wait();
+        }
+        if (cfirst + kStep >= ncols) {  // every column is in registers: the MMAs may go on
           release(acc);
           freed = true;
         }
-        for (int c0 = 0; c0 < ncols; c0 += 64) {
+        for (int c0 = cfirst; c0 < ncols; c0 += kStep) {
           uint32_t wa[16], wb[16];
           pack(va, wa);
           pack(vb, wb);
-          const bool more = c0 + 64 < ncols;
+          const bool more = c0 + kStep < ncols;
           if (more) {
-            tmem_ld_32x32b_x32(tbase + (uint32_t)(c0 + 64), va);
-            tmem_ld_32x32b_x32(tbase + (uint32_t)(c0 + 96), vb);
+            tmem_ld_32x32b_x32(tbase + (uint32_t)(c0 + kStep), va);
+            tmem_ld_32x32b_x32(tbase + (uint32_t)(c0 + kStep + 32), vb);
           }
-          uint8_t* buf = epi + q * 8192 + (nstore & 1u) * 4096u;
-          if (lane == 0) bulk_wait_group_read<1>();  // the store that last used buf has read it
+          uint8_t* buf = epi + ew * (kBufs * 4096) + (nstore % kBufs) * 4096u;
+          // the store that last used buf has read it
+          if (lane == 0) bulk_wait_group_read<kBufs - 1>();
           __syncwarp();
 #pragma unroll
           for (int c = 0; c < 8; ++c) {  // 128-byte swizzle: 16-byte chunk c ^ (row % 8)
@@ -565,14 +597,14 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
           ++nstore;
           if (more) {
             tmem_ld_wait();
-            if (c0 + 128 >= ncols) {  // those were the last columns
+            if (c0 + 2 * kStep >= ncols) {  // those were this warp's last columns
               release(acc);
               freed = true;
             }
           }
         }
       }
-      for (int c0 = 0; MODE != kPWgrad && live && c0 < ncols; c0 += 32) {
+      for (int c0 = grp * 32; MODE != kPWgrad && live && c0 < ncols; c0 += kChunkStep) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tbase + (uint32_t)c0, v);
         tmem_ld_wait();
@@ -584,38 +616,39 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
           const int ucol = routed ? p.ucol_routed : p.ucol_shared;
 #pragma unroll
           for (int it = 0; it < 4; ++it) {
-            const int i = et + it * kEpiThreads;
+            const int i = eg + it * kGrpThreads;
             const int r = i >> 4, cv = i & 15;
-            *reinterpret_cast<uint4*>(epi_g + r * 128 + cv * 8) = gpre[it];
-            *reinterpret_cast<uint4*>(epi_u + r * 128 + cv * 8) = upre[it];
+            *reinterpret_cast<uint4*>(gbuf + r * 128 + cv * 8) = gpre[it];
+            *reinterpret_cast<uint4*>(ubuf + r * 128 + cv * 8) = upre[it];
           }
-          named_bar_sync(1, kEpiThreads);
-          if (c0 + 32 < ncols) load_gu(t, r0, c0 + 32);  // next chunk, in flight meanwhile
+          named_bar_sync(gbar, kGrpThreads);
+          // this group's next chunk, in flight meanwhile
+          if (c0 + kChunkStep < ncols) load_gu(t, r0, c0 + kChunkStep);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (j < nj) {
               const float dh = __uint_as_float(v[j]);
-              const float g = __uint_as_float((uint32_t)epi_g[j * 128 + mrow] << 16);
-              const float u = __uint_as_float((uint32_t)epi_u[j * 128 + mrow] << 16);
+              const float g = __uint_as_float((uint32_t)gbuf[j * 128 + mrow] << 16);
+              const float u = __uint_as_float((uint32_t)ubuf[j * 128 + mrow] << 16);
               const float sg = pb_sigmoid(g);
               const float dg = dh * u * (sg * (1.0f + g * (1.0f - sg)));
               const float du = dh * (g * sg);
-              epi_g[j * 128 + mrow] = __bfloat16_as_ushort(__float2bfloat16_rn(dg));
-              epi_u[j * 128 + mrow] = __bfloat16_as_ushort(__float2bfloat16_rn(du));
+              gbuf[j * 128 + mrow] = __bfloat16_as_ushort(__float2bfloat16_rn(dg));
+              ubuf[j * 128 + mrow] = __bfloat16_as_ushort(__float2bfloat16_rn(du));
             }
           }
-          named_bar_sync(1, kEpiThreads);
-          for (int i = et; i < 32 * 16; i += kEpiThreads) {
+          named_bar_sync(gbar, kGrpThreads);
+          for (int i = eg; i < 32 * 16; i += kGrpThreads) {
             const int r = i >> 4, cv = i & 15;
             if (r < nj) {
               const size_t row = (size_t)(t.row0 + c0 + r) * ldo + r0 + cv * 8;
               *reinterpret_cast<uint4*>(out + row) =
-                  *reinterpret_cast<const uint4*>(epi_g + r * 128 + cv * 8);
+                  *reinterpret_cast<const uint4*>(gbuf + r * 128 + cv * 8);
               *reinterpret_cast<uint4*>(out + row + ucol) =
-                  *reinterpret_cast<const uint4*>(epi_u + r * 128 + cv * 8);
+                  *reinterpret_cast<const uint4*>(ubuf + r * 128 + cv * 8);
             }
           }
-          named_bar_sync(1, kEpiThreads);  // the tile is reused by the next chunk
+          named_bar_sync(gbar, kGrpThreads);  // the tile is reused by the next chunk
         } else {
           // dX for feature r0 + mrow and the tile's token rows, fp32
           const int col = r0 + mrow;
@@ -700,7 +733,7 @@ cudaError_t launch_pb(const CUtensorMap* m, const PBParams& p, int num_sms, cuda
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(block_threads(MODE), 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = attr;
