@@ -136,8 +136,10 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
   extern __shared__ uint8_t dsmem_raw[];
   const uint32_t raw = smem_u32(dsmem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
+  // SwiGLU epilogue staging: one 32-token chunk of u, then of g ([32][64] fp32 each)
   float* up_buf =
       reinterpret_cast<float*>(dsmem_raw + (sbase - raw) + kStages * (kABytes + kBBytes));
+  float* gate_buf = up_buf + 32 * 64;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -388,34 +390,38 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
                     __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
           }
         } else {
-          if (q >= 2) {
+          // the gate lanes (q < 2) stage g, the up lanes (q >= 2) stage u;
+          // then each pair of warps finishes half of the chunk's tokens for
+          // the same 64 features, so all four warps share the SwiGLU and the
+          // stores of h (and, training, of g and u)
+          const int f = frow & 63;  // feature of this lane's accumulator row
+          float* mine = q < 2 ? gate_buf : up_buf;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) up_buf[j * 64 + (frow - 64)] = __uint_as_float(v[j]);
-          }
+          for (int j = 0; j < 32; ++j) mine[j * 64 + f] = __uint_as_float(v[j]);
           named_bar_sync(1, kEpiThreads);
-          if (q < 2) {
-            uint16_t* out = static_cast<uint16_t*>(routed ? p.out_routed : p.out_shared);
-            const int ld = routed ? p.ld_routed : p.ld_shared;
-            const int col = t.ft * 128 + (int)rank * 64 + frow;
+          uint16_t* out = static_cast<uint16_t*>(routed ? p.out_routed : p.out_shared);
+          const int ld = routed ? p.ld_routed : p.ld_shared;
+          const int col = t.ft * 128 + (int)rank * 64 + f;
+          const int jb = q < 2 ? 0 : 16;  // this warp's half of the tokens
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (j < nj) {
-                const float g = __uint_as_float(v[j]);
-                const float h = psilu(g) * up_buf[j * 64 + frow];
-                out[(size_t)(t.row0 + c0 + j) * ld + col] =
-                    __bfloat16_as_ushort(__float2bfloat16_rn(h));
-              }
+          for (int jj = 0; jj < 16; ++jj) {
+            const int j = jb + jj;
+            if (j < nj) {
+              const float h = psilu(gate_buf[j * 64 + f]) * up_buf[j * 64 + f];
+              out[(size_t)(t.row0 + c0 + j) * ld + col] =
+                  __bfloat16_as_ushort(__float2bfloat16_rn(h));
             }
-            uint16_t* gs = routed ? p.g_routed : p.g_shared;
-            uint16_t* us = routed ? p.u_routed : p.u_shared;
-            if (gs != nullptr) {
+          }
+          uint16_t* gs = routed ? p.g_routed : p.g_shared;
+          uint16_t* us = routed ? p.u_routed : p.u_shared;
+          if (gs != nullptr) {
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                if (j < nj) {
-                  const size_t at = (size_t)(t.row0 + c0 + j) * ld + col;
-                  gs[at] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
-                  us[at] = __bfloat16_as_ushort(__float2bfloat16_rn(up_buf[j * 64 + frow]));
-                }
+            for (int jj = 0; jj < 16; ++jj) {
+              const int j = jb + jj;
+              if (j < nj) {
+                const size_t at = (size_t)(t.row0 + c0 + j) * ld + col;
+                gs[at] = __bfloat16_as_ushort(__float2bfloat16_rn(gate_buf[j * 64 + f]));
+                us[at] = __bfloat16_as_ushort(__float2bfloat16_rn(up_buf[j * 64 + f]));
               }
             }
           }
@@ -476,7 +482,7 @@ bool make_map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, 
 
 template <int MODE>
 cudaError_t launch_pair(const CUtensorMap* m, const PairParams& p, int num_sms, cudaStream_t st) {
-  constexpr size_t smem = (size_t)kStages * (kABytes + kBBytes) + 32 * 64 * 4 + 1024;
+  constexpr size_t smem = (size_t)kStages * (kABytes + kBBytes) + 2 * 32 * 64 * 4 + 1024;
   static_assert(smem + sizeof(PCtl) <= 232448, "shared memory budget");
   auto kern = grouped_gemm_pair_kernel<MODE>;
   cudaError_t err =
