@@ -555,3 +555,36 @@ def test_ep_recv_rows_gathers_the_source_tokens():
         rows = O.ep_recv_rows(x, L, r)
         for i, (s, t) in enumerate(L["src_of_row"][r]):
             np.testing.assert_array_equal(rows[i], x[s][t] if s >= 0 else np.zeros(8))
+
+
+@pytest.mark.parametrize("W,align", [(1, 16), (2, 4), (4, 16)])
+def test_ep_exchange_reproduces_the_layer_output(W, align):
+    """Every rank routes its own tokens; the rows move to their owners by the
+    layout, each owner runs its experts segment by segment, and each rank
+    reads its pairs' outputs back by (owner, row) and combines them with its
+    shared experts: the result is forward() of that rank's tokens."""
+    cfg = small_config(T=11, d=32, E=8, k=2, S=1, I=16)
+    base = make_inputs(cfg)
+    host = {n: (v.double().numpy() if torch.is_tensor(v) else v) for n, v in base.items()}
+    xs = [host["x"]] + [make_inputs(cfg, seed=300 + r, weights=False)["x"].double().numpy()
+                        for r in range(1, W)]
+    routes = [O.route(x, host["w_gate"], host["bias"], cfg.k) for x in xs]
+    L = O.ep_layout([r["idx"] for r in routes], cfg.E, align)
+    El = cfg.E // W
+    outs = []
+    for r in range(W):
+        rows = O.ep_recv_rows(xs, L, r)
+        o = np.zeros_like(rows)
+        for le in range(El):
+            a, b = int(L["recv_offsets"][r, le]), int(L["recv_offsets"][r, le + 1])
+            e = r * El + le
+            if b > a:
+                o[a:b] = O.swiglu_expert(rows[a:b], host["w1"][e], host["w3"][e], host["w2"][e])[0]
+        outs.append(o)
+    for s, x in enumerate(xs):
+        y = O.swiglu_expert(x, host["ws1"][0], host["ws3"][0], host["ws2"][0])[0]
+        for p in range(x.shape[0] * cfg.k):
+            t, j = divmod(p, cfg.k)
+            y[t] += routes[s]["w"][t, j] * outs[L["owner"][s][p]][L["row"][s][p]]
+        want = O.forward(dict(host, x=x, T=x.shape[0]), align=align)["y"]
+        np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-12)
