@@ -2,6 +2,8 @@
 // sequence of every entry point declared in include/moe_b200.h.
 #include <cstdint>
 #include <cstring>
+
+#include <cudaTypedefs.h>
 #include <mutex>
 
 #include "../../include/moe_b200.h"
@@ -768,6 +770,47 @@ int moe_ep_combine(const moe_dims* dims, int world, const moe_bf16* const* y_rec
                                        at<float>(ws, L.topk_w),
                                        s.S > 0 ? at<float>(ws, L.y_shared) : nullptr, y,
                                        static_cast<cudaStream_t>(stream)));
+}
+
+int moe_ipc_export(const void* ptr, void* handle, uint64_t* offset) {
+  if (ptr == nullptr || handle == nullptr || offset == nullptr) return MOE_ERR_INVALID_ARG;
+  static PFN_cuMemGetAddressRange_v3020 range = nullptr;
+  if (range == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return MOE_ERR_CUDA;
+    range = reinterpret_cast<PFN_cuMemGetAddressRange_v3020>(fn);
+  }
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (range(&base, &size, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS)
+    return MOE_ERR_CUDA;
+  cudaIpcMemHandle_t h;
+  if (cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base)) != cudaSuccess) return MOE_ERR_CUDA;
+  static_assert(sizeof(h) == 64, "IPC handle size");
+  std::memcpy(handle, &h, sizeof(h));
+  *offset = reinterpret_cast<uint64_t>(ptr) - static_cast<uint64_t>(base);
+  return MOE_OK;
+}
+
+int moe_ipc_open(const void* handle, uint64_t offset, void** ptr) {
+  if (handle == nullptr || ptr == nullptr) return MOE_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  std::memcpy(&h, handle, sizeof(h));
+  void* base = nullptr;
+  if (cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  *ptr = static_cast<char*>(base) + offset;
+  return MOE_OK;
+}
+
+int moe_ipc_close(void* ptr, uint64_t offset) {
+  if (ptr == nullptr) return MOE_ERR_INVALID_ARG;
+  return cudaIpcCloseMemHandle(static_cast<char*>(ptr) - offset) == cudaSuccess ? MOE_OK
+                                                                                 : MOE_ERR_CUDA;
 }
 
 int moe_get_last_device_status(void* stream) {

@@ -32,6 +32,7 @@ EXPORTED = (
     "moe_dense_workspace_size", "moe_dense_swiglu",
     "moe_ep_recv_capacity", "moe_ep_workspace_size", "moe_ep_layout_of", "moe_ep_route",
     "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine",
+    "moe_ipc_export", "moe_ipc_open", "moe_ipc_close",
 )
 
 
@@ -112,6 +113,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_ep_dispatch": (I, [P, I, I, V, V, V, V, Z, V]),
         "moe_ep_experts": (I, [P, I, V, V, V, V, V, V, V, V, V, V, Z, V]),
         "moe_ep_combine": (I, [P, I, V, V, V, Z, V]),
+        "moe_ipc_export": (I, [V, V, ctypes.POINTER(ctypes.c_uint64)]),
+        "moe_ipc_open": (I, [V, ctypes.c_uint64, ctypes.POINTER(ctypes.c_void_p)]),
+        "moe_ipc_close": (I, [V, ctypes.c_uint64]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -427,6 +431,28 @@ def ep_combine(dm, world, y_recv, y, workspace, stream=None):
     _check(load().moe_ep_combine(ctypes.byref(dm), int(world), _ptr(y_recv), _ptr(y),
                                  _ptr(workspace), workspace.numel(), _stream(stream)),
            "moe_ep_combine")
+
+
+def ipc_export(t: torch.Tensor) -> tuple[bytes, int]:
+    """CUDA IPC handle (64 bytes) of the allocation holding tensor t, and t's
+    byte offset inside it."""
+    h = ctypes.create_string_buffer(64)
+    off = ctypes.c_uint64(0)
+    _check(load().moe_ipc_export(_ptr(t), h, ctypes.byref(off)), "moe_ipc_export")
+    return h.raw, int(off.value)
+
+
+def ipc_open(handle: bytes, offset: int) -> int:
+    """Device address, in this process, of another process's exported tensor."""
+    if len(handle) != 64:
+        raise ValueError("an IPC handle is 64 bytes")
+    p = ctypes.c_void_p(0)
+    _check(load().moe_ipc_open(handle, ctypes.c_uint64(offset), ctypes.byref(p)), "moe_ipc_open")
+    return int(p.value)
+
+
+def ipc_close(ptr: int, offset: int) -> None:
+    _check(load().moe_ipc_close(ctypes.c_void_p(ptr), ctypes.c_uint64(offset)), "moe_ipc_close")
 
 
 def ep_workspace_views(dm: MoeDims, world: int, ws: torch.Tensor) -> dict:

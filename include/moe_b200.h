@@ -453,6 +453,24 @@ int moe_ep_combine(const moe_dims* dims, int world, const moe_bf16* const* y_rec
                    moe_bf16* y, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * CUDA IPC of the expert-parallel buffers (receive buffers, counts) between
+ * the processes of one node, one process per GPU.
+ *
+ * moe_ipc_export -- ptr: a device address inside an allocation of this
+ *   process made by cudaMalloc (PyTorch's default allocator); writes the
+ *   allocation's 64-byte IPC handle to `handle` and ptr's offset inside the
+ *   allocation to `offset`.
+ * moe_ipc_open -- maps another process's allocation on the current device
+ *   (peer access enabled lazily) and returns the address of handle + offset
+ *   in *ptr.  A process cannot open its own handles (CUDA rejects them).
+ * moe_ipc_close -- unmaps what moe_ipc_open returned (same offset).
+ * Return MOE_OK, MOE_ERR_INVALID_ARG (null pointer) or MOE_ERR_CUDA.
+ * ---------------------------------------------------------------------- */
+int moe_ipc_export(const void* ptr, void* handle, uint64_t* offset);
+int moe_ipc_open(const void* handle, uint64_t offset, void** ptr);
+int moe_ipc_close(void* ptr, uint64_t offset);
+
+/* ------------------------------------------------------------------------
  * Device status and bounded waits.
  *
  * moe_get_last_device_status: synchronises `stream`, returns the first error

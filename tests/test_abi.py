@@ -163,6 +163,20 @@ def test_expert_parallel_sizes_and_rejects_on_host(lib):
                               None) == M.MOE_ERR_WORKSPACE
 
 
+def test_ipc_calls_rejected_on_host(lib):
+    h = ctypes.create_string_buffer(64)
+    off = ctypes.c_uint64(0)
+    ptr = ctypes.c_void_p(0)
+    assert lib.moe_ipc_export(None, h, ctypes.byref(off)) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_ipc_export(ctypes.c_void_p(1 << 20), None, ctypes.byref(off)) == \
+        M.MOE_ERR_INVALID_ARG
+    assert lib.moe_ipc_open(None, 0, ctypes.byref(ptr)) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_ipc_open(h, 0, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_ipc_close(None, 0) == M.MOE_ERR_INVALID_ARG
+    with pytest.raises(ValueError):
+        M.ipc_open(b"short", 0)
+
+
 def test_status_strings(lib):
     for s in (0, -1, -2, -3, -4, -5):
         assert M.status_string(s) != "unknown status"

@@ -142,3 +142,53 @@ def test_two_rank_weight_gradient_allreduce_on_gloo():
     for r in range(world):
         assert all(v == 3.0 for v in res[r]["weights"])   # 1 + 2 on every rank
         assert res[r]["dx"] == float(r + 1)
+
+
+def _ep_exchange_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    from fine_grained_moe_fp32_b200 import ep_dist
+
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # fake handles: byte 0 names the owner's allocation; "x_recv" and
+        # "y_recv" share one allocation (one handle, two offsets), as the
+        # caching allocator may arrange; the fake opener's base shows the owner
+        local = {"x_recv": (bytes([rank]) * 64, 16 * rank, 1000 + rank),
+                 "y_recv": (bytes([rank]) * 64, 16 * rank + 4096, 1100 + rank),
+                 "counts": (bytes([rank + 100]) * 64, 8, 2000 + rank)}
+        calls = []
+
+        def opener(h):
+            calls.append(h[0])
+            return 5000 + 100 * h[0]
+
+        addrs, opened = ep_dist.exchange_pointers(local, opener=opener)
+        out[rank] = {"addrs": addrs, "opened": opened, "calls": calls}
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_ep_pointer_exchange_on_gloo(world):
+    """Every rank gets every buffer's address in rank order: its own as it
+    is, a peer's as the base of that peer's allocation (opened once per
+    distinct handle) plus the buffer's offset."""
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.start_processes(_ep_exchange_worker, args=(world, port, out), nprocs=world,
+                           join=True, start_method="spawn")
+        res = dict(out)
+    for r in range(world):
+        a = res[r]["addrs"]
+        for s in range(world):
+            if s == r:
+                assert (a["x_recv"][s], a["y_recv"][s], a["counts"][s]) == \
+                    (1000 + r, 1100 + r, 2000 + r)
+            else:
+                assert a["x_recv"][s] == 5000 + 100 * s + 16 * s
+                assert a["y_recv"][s] == 5000 + 100 * s + 16 * s + 4096
+                assert a["counts"][s] == 5000 + 100 * (s + 100) + 8
+        peers = [s for s in range(world) if s != r]
+        assert sorted(res[r]["calls"]) == sorted(peers + [s + 100 for s in peers])
+        assert len(res[r]["opened"]) == 2 * (world - 1)
