@@ -44,7 +44,7 @@ def _worker(rank, world, port, out):
 def test_two_rank_replicas_on_gloo():
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.start_processes(_worker, args=(world, port, out), nprocs=world, join=True,
                            start_method="spawn")
@@ -100,7 +100,7 @@ def _loads_worker(rank, world, port, out):
 def test_two_rank_bias_step_uses_global_loads_on_gloo():
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.start_processes(_loads_worker, args=(world, port, out), nprocs=world, join=True,
                            start_method="spawn")
@@ -134,7 +134,7 @@ def _grads_worker(rank, world, port, out):
 def test_two_rank_weight_gradient_allreduce_on_gloo():
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.start_processes(_grads_worker, args=(world, port, out), nprocs=world, join=True,
                            start_method="spawn")
@@ -174,7 +174,7 @@ def test_ep_pointer_exchange_on_gloo(world):
     is, a peer's as the base of that peer's allocation (opened once per
     distinct handle) plus the buffer's offset."""
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.start_processes(_ep_exchange_worker, args=(world, port, out), nprocs=world,
                            join=True, start_method="spawn")

@@ -220,7 +220,7 @@ def _stage_worker(r, P, V, M, overlap, port, out):
 def test_processes_running_the_schedule_reproduce_sequential_gradients(P, V, overlap):
     M = 2 * P
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.start_processes(_stage_worker, args=(P, V, M, overlap, port, out), nprocs=P,
                            join=True, start_method="spawn")
