@@ -1,11 +1,12 @@
 """Pipeline schedule of the training step: interleaved 1F1B with the MoE
 all-to-all overlapped (dots.llm1 Technical Report, Method / Key claims,
-systems paragraph: a variant of interleaved 1F1B that overlaps the MoE
-all-to-all with computation in the steady phase, costs one more warm-up step
-and needs no extra activation memory; "How dots.llm1's 14B MoE Architecture
-Matches 72B LLM Performance", Computational Infrastructure Innovations).
+systems paragraph, and "How dots.llm1's 14B MoE Architecture Matches 72B LLM
+Performance", Computational Infrastructure Innovations).  What the pages fix:
+in the steady state the expert all-to-all is hidden behind the math of
+another pass; the price is a single additional warm-up pass; the activation
+footprint stays that of the plain schedule.
 
-The pages state those properties, not the schedule.  The reading built here:
+The pages give those properties, not the schedule.  The reading built here:
 
 * P pipeline stages, V model chunks per stage (chunk v of stage r is the
   layer block v*P + r, so a microbatch visits stages 0..P-1 V times), M
