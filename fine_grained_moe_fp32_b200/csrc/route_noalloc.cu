@@ -13,7 +13,9 @@
 // code cannot use the array's name as a device address, so on the first call
 // on each device (with that device current) its address is looked up with
 // cudaGetSymbolAddress and cached; that first call should therefore come
-// before any stream capture.  Every call shares the array: the router
+// before any stream capture.  The cache lives as long as the process: after a
+// cudaDeviceReset the cached address is stale, and the library must not be
+// called again in that process.  Every call shares the array: the router
 // overwrites all of the partials it later reads, so nothing has to start at
 // zero, but two calls that overlap on the GPU (different streams, or
 // different host threads on one device) race on it.

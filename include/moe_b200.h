@@ -107,14 +107,19 @@ int moe_route(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
  * holds until the process exits.
  *
  * Arguments and results are those of moe_route (same kernels, bit-identical
- * output).  Shapes whose partials need more than 16 MiB
- * (moe_route_workspace_size(dims) > 16 MiB, e.g. E = 128 beyond ~30k
- * tokens) are rejected with MOE_ERR_WORKSPACE before anything is launched.
+ * output).  The split-K planner keeps the partials within 16 MiB whenever one
+ * split fits, so a shape is rejected (MOE_ERR_WORKSPACE, nothing launched)
+ * exactly when one split alone needs more: T * E * 4 bytes > 16 MiB, i.e.
+ * T * E > 4194304 (T > 32768 at E = 128).
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
- * capture.  All calls share the array: it needs no clearing (every partial
- * read is written first in the same call), but calls that overlap on the GPU
- * (other streams, other host threads on the same device) race on it.
+ * capture.  The address is cached for the life of the process: after a
+ * cudaDeviceReset the cached address (and the library's device status word
+ * address, cached the same way) is stale, so do not call the library again
+ * in that process after a reset.  All calls share the array: it needs no
+ * clearing (every partial read is written first in the same call), but calls
+ * that overlap on the GPU (other streams, other host threads on the same
+ * device) race on it.
  * ---------------------------------------------------------------------- */
 int moe_route_noalloc(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
                       const float* bias, float* probs, int32_t* topk_idx,

@@ -180,3 +180,16 @@ def test_ipc_calls_rejected_on_host(lib):
 def test_status_strings(lib):
     for s in (0, -1, -2, -3, -4, -5):
         assert M.status_string(s) != "unknown status"
+
+
+def test_no_alloc_route_rejects_shapes_beyond_its_scratch(lib):
+    """The size check of moe_route_noalloc comes before any pointer is used or
+    any CUDA call is made: one split of T * E fp32 partial logits above the
+    built-in 16 MiB is rejected, one that fits is not rejected for size."""
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced
+    over = M.dims(T=32769, d=5120, E=128, k=6, I=1408, n_shared=2, align=16)
+    assert 32769 * 128 * 4 > (16 << 20)
+    assert lib.moe_route_noalloc(ctypes.byref(over), fake, fake, None, None, fake, fake,
+                                 None) == M.MOE_ERR_WORKSPACE
+    assert M.route_workspace_size(M.dims(T=32768, d=5120, E=128, k=6, I=1408, n_shared=2,
+                                         align=16)) <= (16 << 20)
