@@ -199,7 +199,7 @@ def gemm_units(cfg, T, counts):
     touched = int((counts > 0).sum())
     rows = T * k
     g1_bytes = (touched + S) * 2 * I * d * 2 + (rows + T) * d * 2 + (rows + T * S) * I * 2
-    g2_bytes = (touched + S) * d * I * 2 + (rows + T * S) * I * 2 + rows * d * 2 + T * d * 4
+    g2_bytes = (touched + S) * d * I * 2 + (rows + T * S) * I * 2 + rows * d * 4 + T * d * 4
     g1_flops = 2 * (rows * 2 * I + T * 2 * S * I) * d
     g2_flops = 2 * (rows * I + T * S * I) * d
     return {"touched_experts": touched, "gemm_gate_up_swiglu": (g1_bytes, g1_flops),
@@ -266,6 +266,8 @@ def run_reference(args):
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = make_inputs(cfg, device=dev)
     host = {k: (v.detach().cpu() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    from oracle import moe_oracle as O
+    touched = len(np.unique(O.route(host["x"], host["w_gate"], host["bias"], cfg.k)["idx"]))
     n = args.ref_tokens
     for _ in range(args.warmup):
         oracle_sample(host, n, seed=1)
@@ -280,8 +282,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
-                   "S": cfg.S, "I": cfg.I},
+        "config": config_dict(cfg, args.gpus, args.align, touched),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_threads(),
                          "kind": "oracle",
                          "sample": f"{nt} seeded tokens of the T={cfg.T} batch per step, "
@@ -293,19 +294,44 @@ def run_reference(args):
     return 0
 
 
-def run_ours(args):
+NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}   # B200 spec sheet, dense bf16
+EXTRA_CONFIGS = (2, 3, 4)   # measured beside the headline decode line, same K and W
+
+
+def layer_units(cfg, T, counts, train):
+    """Algorithmic work of one whole step of the layer: the bytes it must move
+    (every touched routed expert's and the shared experts' weights, the fp32
+    gate, tokens in and out) and the tensor-core flops (3 contractions of
+    2*d*I per expert row; the backward doubles them)."""
+    d, I, S, k, E = cfg.d, cfg.I, cfg.S, cfg.k, cfg.E
+    touched = int((counts > 0).sum())
+    bytes_ = (touched + S) * 3 * d * I * 2 + E * d * 4 + 2 * T * d * 2
+    flops = 2 * 3 * d * I * (T * k + T * S) * (3 if train else 1)
+    return bytes_, flops
+
+
+def config_dict(cfg, world, align, touched):
+    c = {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
+         "S": cfg.S, "I": cfg.I, "align": align, "router": "fp32",
+         "parallelism": f"dp{world} (replicas, no collective)",
+         "l2": "inputs larger than L2: the step streams the expert weights "
+               f"({(touched + cfg.S) * 3 * cfg.I * cfg.d * 2 / 1e9:.2f} GB)"}
+    if cfg.grad:
+        c["step"] = ("forward (training, keeps g/u) + backward + sequence-wise balance "
+                     f"statistics (seq_len {math.gcd(cfg.T, BALANCE_SEQ)}) + bias step"
+                     + (" + weight-gradient all-reduce and summed expert loads (NCCL)"
+                        if world > 1 else ""))
+        if world > 1:
+            c["parallelism"] = f"dp{world} (weight gradients all-reduced)"
+    return c
+
+
+def measure(cfg, args, dev, world, rank, local):
+    """Time one workload on this rank's GPU: W warm-up steps, an untimed pass
+    with every phase bracketed by events, K timed steps (device-resident
+    inputs), K end-to-end steps through the public API with host copies.
+    Returns plain numbers only, so every device tensor is freed on return."""
     from fine_grained_moe_fp32_b200 import moe as M
-    world, rank, local = dist_setup()
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-    cfg = workload(args)
     T = cfg.T
     inp = make_inputs(cfg, device=dev, seed=0, weights=True)
     if world > 1:  # own token batch per rank
@@ -342,14 +368,13 @@ def run_ours(args):
         def step(xin, yout, evs=None, dyin=None, dxout=None):
             layer(xin, yout)
     n_events = 13 if train else 6
-    phase_names = M.PHASES + (M.BWD_PHASES if train else ())
 
     for _ in range(args.warmup):
         step(x, y)
     torch.cuda.synchronize(dev)
     st = M.device_status()
     if st != M.MOE_OK:
-        raise SystemExit(f"device status after warm-up: {M.status_string(st)}")
+        raise SystemExit(f"{cfg.name}: device status after warm-up: {M.status_string(st)}")
     views = M.workspace_views(layer.dims(T), layer.train_workspace(T) if train
                               else layer.workspace(T))
     counts = views["counts"].cpu().numpy()
@@ -414,7 +439,7 @@ def run_ours(args):
     clocks = sampler.stop(t0, t1)
     st = M.device_status()
     if st != M.MOE_OK:
-        raise SystemExit(f"device status after timing: {M.status_string(st)}")
+        raise SystemExit(f"{cfg.name}: device status after timing: {M.status_string(st)}")
     ms_local = start.elapsed_time(end)
     ms = max_over_ranks(ms_local, world, dev)
     value = whole_job_value(world, T, args.steps, ms)
@@ -496,46 +521,106 @@ def run_ours(args):
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak}
     roof["kernel"] = dom
+    roof["kernel_ms"] = dom_ms
     roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if hbm_bound else 'bf16_tflops'})"
     roof["traffic"] = load_traffic(dom, cfg.name)
     roof["algorithmic_per_launch"] = bytes_ if hbm_bound else flops
+    # ---- the whole step against the same two ceilings (measured and nominal)
+    lbytes, lflops = layer_units(cfg, T, counts, train)
+    step_s = ms / args.steps / 1e3   # every rank does one step's work in this time
+    key = "hbm_gbs" if hbm_bound else "bf16_tflops"
+    lach = (lbytes / step_s / 1e9) if hbm_bound else (lflops / step_s / 1e12)
+    roof["layer"] = {"bound": "hbm" if hbm_bound else "tensor", "achieved": lach,
+                     "unit": "GB/s" if hbm_bound else "TFLOP/s",
+                     "algorithmic_per_step": lbytes if hbm_bound else lflops,
+                     "frac_measured": lach / peaks[key],
+                     "frac_nominal": lach / NOMINAL_PEAKS[key],
+                     "nominal_peak": NOMINAL_PEAKS[key]}
+    res = {"value": value, "ms_per_step": ms / args.steps, "roofline": roof,
+           "phases_ms": {k: round(v, 4) for k, v in phase_ms.items()}, "clocks": clocks,
+           "e2e": {"value": e2e_value, "unit": "tokens/s",
+                   "h2d_bytes_per_step": T * cfg.d * 2 * (2 if train else 1),
+                   "d2h_bytes_per_step": T * cfg.d * 2},
+           "gpu_launches": (forward_kernels(T) + (BWD_KERNELS + BALANCE_KERNELS if train else 0))
+           * args.steps,
+           "config": config_dict(cfg, world, args.align, units["touched_experts"]),
+           "n_phase": n_phase}
+    if train:
+        res["train_tflop_per_step"] = sum(train_gemm_flops(cfg, T).values()) / 1e12
+    return res
 
+
+def cpu_baseline_full(cfg):
+    """The fp64 oracle on a whole batch of the workload (every token, the
+    oracle's own permutation path), timed on this host's cores."""
+    from oracle import moe_oracle as O
+    inp = make_inputs(cfg, device="cpu")
+    host = {k: (v.detach() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    t0 = time.perf_counter()
+    O.forward(host)
+    return cfg.T, time.perf_counter() - t0
+
+
+def run_ours(args):
+    world, rank, local = dist_setup()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    cfg = workload(args)
+    r = measure(cfg, args, dev, world, rank, local)
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "metric": METRIC, "value": r["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights; random-init layer)",
-        "config": {"workload": cfg.name, "T": T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
-                   "S": cfg.S, "I": cfg.I, "align": args.align, "router": "fp32",
-                   "parallelism": f"dp{world} (replicas, no collective)",
-                   "l2": "inputs larger than L2: the step streams the expert weights "
-                         f"({(units['touched_experts'] + cfg.S) * 3 * cfg.I * cfg.d * 2 / 1e9:.2f} GB)"},
-        "roofline": roof,
-        "phases_ms": {k: round(v, 4) for k, v in phase_ms.items()},
-        "phases_ms_source": f"untimed pass of {n_phase} steps with every phase bracketed by "
-                            "events; the timed region brackets only the roofline kernel",
-        "clocks": clocks,
-        "e2e": {"value": e2e_value, "unit": "tokens/s",
-                "h2d_bytes_per_step": T * cfg.d * 2 * (2 if train else 1),
-                "d2h_bytes_per_step": T * cfg.d * 2},
-        "gpu_launches": (forward_kernels(T) + (BWD_KERNELS + BALANCE_KERNELS if train else 0))
-        * args.steps,
+        "config": r["config"],
+        "roofline": r["roofline"],
+        "phases_ms": r["phases_ms"],
+        "phases_ms_source": f"untimed pass of {r['n_phase']} steps with every phase bracketed "
+                            "by events; the timed region brackets only the roofline kernel",
+        "clocks": r["clocks"], "e2e": r["e2e"], "gpu_launches": r["gpu_launches"],
     }
-    if train:
-        line["config"]["step"] = ("forward (training, keeps g/u) + backward + sequence-wise "
-                                  f"balance statistics (seq_len {seq_len}) + bias step"
-                                  + (" + weight-gradient all-reduce and summed expert loads "
-                                     "(NCCL)" if world > 1 else ""))
-        if world > 1:
-            line["config"]["parallelism"] = f"dp{world} (weight gradients all-reduced)"
-        line["train_tflop_per_step"] = sum(train_gemm_flops(cfg, T).values()) / 1e12
+    if "train_tflop_per_step" in r:
+        line["train_tflop_per_step"] = r["train_tflop_per_step"]
+    shrunk = bool(args.experts or args.tokens or args.inter)
+    if world == 1 and args.config == 1 and not shrunk and not args.no_extra_configs:
+        # the prefill and training workloads, each timed like the headline
+        extra = {}
+        for c in EXTRA_CONFIGS:
+            torch.cuda.empty_cache()
+            rc = measure(CONFIGS[c], args, dev, world, rank, local)
+            rc.pop("n_phase")
+            extra[CONFIGS[c].name] = {"tokens_per_s": rc.pop("value"), **rc}
+            line["gpu_launches"] += rc["gpu_launches"]
+        line["configs"] = extra
+        line["configs_note"] = ("the prefill and fwd+bwd workloads, each timed like the "
+                                f"headline ({args.warmup} warm-up, {args.steps} timed steps, "
+                                "CUDA events, clocks sampled); gpu_launches above counts "
+                                "their launches too")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n, dt = oracle_sample(inp, args.cpu_tokens)
-        line["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": cpu_threads(),
-                                "kind": "oracle",
-                                "sample": f"{n} seeded tokens of the T={T} batch, fp64 numpy "
-                                          f"oracle ({'forward + backward' if train else 'forward'}"
-                                          f"), {dt:.1f} s"}
+        if cfg.T <= 256 and not cfg.grad:
+            n, dt = cpu_baseline_full(cfg)
+            n0, dt0 = cpu_baseline_full(CONFIGS[0])
+            line["cpu_baseline"] = {
+                "value": n / dt, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+                "sample": f"the whole T={n} batch of {cfg.name} through the fp64 numpy oracle "
+                          f"(route, permute, 128 experts, shared, combine): {dt:.1f} s",
+                "tiny_full": {"workload": CONFIGS[0].name, "value": n0 / dt0,
+                              "unit": "tokens/s", "seconds": dt0}}
+        else:
+            inp = make_inputs(cfg, device=dev)
+            n, dt = oracle_sample(inp, args.cpu_tokens)
+            line["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": cpu_threads(),
+                                    "kind": "oracle",
+                                    "sample": f"{n} seeded tokens of the T={cfg.T} batch, fp64 "
+                                              f"numpy oracle ({'forward + backward' if cfg.grad else 'forward'}"
+                                              f"), {dt:.1f} s"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -837,8 +922,11 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--align", type=int, default=16)
     ap.add_argument("--cpu-tokens", type=int, default=32)
-    ap.add_argument("--ref-tokens", type=int, default=4)
+    ap.add_argument("--ref-tokens", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra-configs", action="store_true",
+                    help="time only --config (the default run adds the prefill and fwd+bwd "
+                         "workloads to the headline decode line)")
     ap.add_argument("--experts", type=int, default=0, help="shrink E (profiling cases)")
     ap.add_argument("--tokens", type=int, default=0, help="override T (profiling cases)")
     ap.add_argument("--inter", type=int, default=0, help="override I (profiling cases)")

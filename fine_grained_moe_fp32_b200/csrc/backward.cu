@@ -29,7 +29,7 @@ constexpr int kMaxVecPerThread = 8;  // d <= 8 * 8 * 128 = 8192
 // One CTA per token.  The dot products are reduced in a fixed order (per
 // thread, then warp butterfly, then warps in order), so dw is deterministic.
 __global__ void __launch_bounds__(kCbThreads)
-combine_bwd_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ y_perm,
+combine_bwd_kernel(const uint16_t* __restrict__ dy, const float* __restrict__ y_perm,
                    const int32_t* __restrict__ row_of, const float* __restrict__ topk_w,
                    uint16_t* __restrict__ dy_perm, float* __restrict__ dw, int d, int k,
                    int64_t cap) {
@@ -47,20 +47,20 @@ combine_bwd_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__
     const float w = topk_w[(size_t)t * k + j];
     float part = 0.f;
     if (r >= 0 && r < cap) {
-      const uint4* yr = reinterpret_cast<const uint4*>(y_perm + (size_t)r * d);
+      const float4* yr = reinterpret_cast<const float4*>(y_perm + (size_t)r * d);
       uint4* out = reinterpret_cast<uint4*>(dy_perm + (size_t)r * d);
 #pragma unroll
       for (int i = 0; i < kMaxVecPerThread; ++i) {
         const int v = threadIdx.x + i * kCbThreads;
         if (v < nv) {
-          const uint4 yv = yr[v];
+          const float4 ya = yr[2 * v], yb = yr[2 * v + 1];
           const uint32_t gw[4] = {g[i].x, g[i].y, g[i].z, g[i].w};
-          const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
+          const float yv[8] = {ya.x, ya.y, ya.z, ya.w, yb.x, yb.y, yb.z, yb.w};
           uint32_t o[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            part = fmaf(bf16lo(gw[q]), bf16lo(yw[q]), part);
-            part = fmaf(bf16hi(gw[q]), bf16hi(yw[q]), part);
+            part = fmaf(bf16lo(gw[q]), yv[2 * q], part);
+            part = fmaf(bf16hi(gw[q]), yv[2 * q + 1], part);
             o[q] = pack_bf16(w * bf16lo(gw[q]), w * bf16hi(gw[q]));
           }
           out[v] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -311,10 +311,12 @@ __global__ void sum_splits_kernel(const float* __restrict__ part, int splits, in
   out[i] = (float)s;
 }
 
+// dx [T, d]: the fp32 sum, rounded once to bf16, or kept in fp32 (F32).
+template <bool F32>
 __global__ void __launch_bounds__(kCbThreads)
 unpermute_bwd_kernel(const float* __restrict__ dx_shared, const float* __restrict__ dx_router,
                      const float* __restrict__ dx_perm, const int32_t* __restrict__ row_of,
-                     uint16_t* __restrict__ dx, int d, int k, int64_t cap) {
+                     void* __restrict__ dx, int d, int k, int64_t cap) {
   const int t = blockIdx.x;
   __shared__ int rows[8];
   if (threadIdx.x < k) {
@@ -345,10 +347,17 @@ unpermute_bwd_kernel(const float* __restrict__ dx_shared, const float* __restric
       acc[0] += p0.x; acc[1] += p0.y; acc[2] += p0.z; acc[3] += p0.w;
       acc[4] += p1.x; acc[5] += p1.y; acc[6] += p1.z; acc[7] += p1.w;
     }
-    uint32_t o[4];
+    if (F32) {
+      float4* o = reinterpret_cast<float4*>(static_cast<float*>(dx) + (size_t)t * d) + 2 * v;
+      o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    } else {
+      uint32_t o[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) o[q] = pack_bf16(acc[2 * q], acc[2 * q + 1]);
-    reinterpret_cast<uint4*>(dx + (size_t)t * d)[v] = make_uint4(o[0], o[1], o[2], o[3]);
+      for (int q = 0; q < 4; ++q) o[q] = pack_bf16(acc[2 * q], acc[2 * q + 1]);
+      reinterpret_cast<uint4*>(static_cast<uint16_t*>(dx) + (size_t)t * d)[v] =
+          make_uint4(o[0], o[1], o[2], o[3]);
+    }
   }
 }
 
@@ -398,8 +407,12 @@ cudaError_t launch_backward_misc_post(const Shape& s, const BackwardMiscArgs& a,
     sum_splits_kernel<<<(unsigned)ceil_div(n, 256), 256, 0, st>>>(a.dwg_partials, splits, n,
                                                                    a.dw_gate);
   }
-  unpermute_bwd_kernel<<<s.T, kCbThreads, 0, st>>>(a.dx_shared, a.dx_router, a.dx_perm, a.row_of,
-                                                   a.dx, s.d, s.k, s.cap);
+  if (a.dx_f32)
+    unpermute_bwd_kernel<true><<<s.T, kCbThreads, 0, st>>>(a.dx_shared, a.dx_router, a.dx_perm,
+                                                           a.row_of, a.dx, s.d, s.k, s.cap);
+  else
+    unpermute_bwd_kernel<false><<<s.T, kCbThreads, 0, st>>>(a.dx_shared, a.dx_router, a.dx_perm,
+                                                            a.row_of, a.dx, s.d, s.k, s.cap);
   return cudaGetLastError();
 }
 

@@ -6,9 +6,11 @@
 //
 //   y[t] = y_shared[t] + sum_{j < k} w[t, j] * y_perm[row_of[t*k + j]]
 //
-// fp32 accumulation, slot j in ascending order, one rounding to bf16.  CTA
-// (t, b) covers 16-byte vectors (8 bf16) b*128 .. b*128+127 of token t, one
-// per thread, with the k routed rows' loads all issued before the sum.
+// The routed outputs y_perm are fp32 (the down GEMM's accumulators, not
+// rounded), so the only rounding of y is the final one.  fp32 accumulation,
+// slot j in ascending order.  CTA (t, b) covers 8-element groups
+// b*128 .. b*128+127 of token t, one per thread (two 16-byte loads per
+// routed row), with the k routed rows' loads all issued before the sum.
 #include <cuda_bf16.h>
 
 #include "moe_internal.h"
@@ -19,21 +21,23 @@ namespace {
 constexpr int kThreads = 128;
 constexpr int kMaxK = 8;
 
-__device__ __forceinline__ void add_bf16x8(float (&acc)[8], uint4 v, float w) {
-  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    acc[2 * i] = fmaf(w, __uint_as_float(u[i] << 16), acc[2 * i]);
-    acc[2 * i + 1] = fmaf(w, __uint_as_float(u[i] & 0xFFFF0000u), acc[2 * i + 1]);
-  }
+__device__ __forceinline__ void add_f32x8(float (&acc)[8], float4 a, float4 b, float w) {
+  acc[0] = fmaf(w, a.x, acc[0]);
+  acc[1] = fmaf(w, a.y, acc[1]);
+  acc[2] = fmaf(w, a.z, acc[2]);
+  acc[3] = fmaf(w, a.w, acc[3]);
+  acc[4] = fmaf(w, b.x, acc[4]);
+  acc[5] = fmaf(w, b.y, acc[5]);
+  acc[6] = fmaf(w, b.z, acc[6]);
+  acc[7] = fmaf(w, b.w, acc[7]);
 }
 
 // Where slot j of token t lives: its row of this rank's segment buffer.
 struct LocalRows {
-  const uint16_t* y_perm;
+  const float* y_perm;
   const int32_t* row_of;
   int64_t cap;
-  __device__ const uint16_t* row(size_t p, int d) const {
+  __device__ const float* row(size_t p, int d) const {
     const int r = row_of[p];
     return (r >= 0 && r < cap) ? y_perm + (size_t)r * d : nullptr;
   }
@@ -42,15 +46,15 @@ struct LocalRows {
 // Expert parallel: the row the dispatch wrote into the owner's receive
 // buffer, read back from there (peer loads when the owner is another GPU).
 struct OwnerRows {
-  const uint16_t* const* y_recv;
+  const float* const* y_recv;
   const int32_t* topk_idx;
   const int32_t* remote_row;
   int E, El;
   int64_t cap;
-  __device__ const uint16_t* row(size_t p, int d) const {
+  __device__ const float* row(size_t p, int d) const {
     const int e = topk_idx[p], r = remote_row[p];
     if (e < 0 || e >= E || r < 0 || r >= cap) return nullptr;
-    const uint16_t* b = y_recv[e / El];
+    const float* b = y_recv[e / El];
     return (reinterpret_cast<uintptr_t>(b) & 15) ? nullptr : b + (size_t)r * d;
   }
 };
@@ -60,7 +64,7 @@ __global__ void __launch_bounds__(kThreads)
 combine_kernel(Rows src, const float* __restrict__ topk_w, const float* __restrict__ y_shared,
                uint16_t* __restrict__ y, int d, int k) {
   const int t = blockIdx.x;
-  __shared__ const uint16_t* rows[kMaxK];
+  __shared__ const float* rows[kMaxK];
   __shared__ float ws[kMaxK];
   if (threadIdx.x < k) {
     rows[threadIdx.x] = src.row((size_t)t * k + threadIdx.x, d);
@@ -80,13 +84,18 @@ combine_kernel(Rows src, const float* __restrict__ topk_w, const float* __restri
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
     }
-    uint4 val[kMaxK];
+    float4 va[kMaxK], vb[kMaxK];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (j < k && rows[j] != nullptr) {
+        const float4* r = reinterpret_cast<const float4*>(rows[j]) + 2 * v;
+        va[j] = __ldg(r);
+        vb[j] = __ldg(r + 1);
+      }
+    }
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j)
-      if (j < k && rows[j] != nullptr) val[j] = __ldg(reinterpret_cast<const uint4*>(rows[j]) + v);
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j)
-      if (j < k && rows[j] != nullptr) add_bf16x8(acc, val[j], ws[j]);
+      if (j < k && rows[j] != nullptr) add_f32x8(acc, va[j], vb[j], ws[j]);
     uint32_t o[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -99,7 +108,7 @@ combine_kernel(Rows src, const float* __restrict__ topk_w, const float* __restri
 
 }  // namespace
 
-cudaError_t launch_combine(const Shape& s, const uint16_t* y_perm, const int32_t* row_of,
+cudaError_t launch_combine(const Shape& s, const float* y_perm, const int32_t* row_of,
                            const float* topk_w, const float* y_shared, uint16_t* y,
                            cudaStream_t st) {
   if (s.T == 0) return cudaSuccess;
@@ -109,7 +118,7 @@ cudaError_t launch_combine(const Shape& s, const uint16_t* y_perm, const int32_t
   return cudaGetLastError();
 }
 
-cudaError_t launch_ep_combine(const Shape& s, int world, const uint16_t* const* y_recv,
+cudaError_t launch_ep_combine(const Shape& s, int world, const float* const* y_recv,
                               const int32_t* topk_idx, const int32_t* remote_row, int64_t cap,
                               const float* topk_w, const float* y_shared, uint16_t* y,
                               cudaStream_t st) {

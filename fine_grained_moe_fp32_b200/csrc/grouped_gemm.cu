@@ -62,12 +62,13 @@ struct GemmParams {
   void* out_shared;
   int ld_shared;
   int shared_f32;
+  int routed_f32;  // down GEMM: routed rows stored in fp32 (else bf16)
   // gate/up GEMM only, training: also store the pre-activations g = W1 x and
-  // u = W3 x (bf16, same layout as h) for the backward pass; null = skip
-  uint16_t* g_routed;
-  uint16_t* u_routed;
-  uint16_t* g_shared;
-  uint16_t* u_shared;
+  // u = W3 x (fp32, same layout as h) for the backward pass; null = skip
+  float* g_routed;
+  float* u_routed;
+  float* g_shared;
+  float* u_shared;
   unsigned int* status;
   uint64_t wait_limit_ns;
 };
@@ -352,7 +353,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r,
         const int nj = min(32, ti.nrows - c0);
         if (MODE == kDown) {
           const int col = ti.ft * 128 + frow;
-          if (routed) {
+          if (routed && p.routed_f32) {
+            float* out = static_cast<float*>(p.out_routed);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nj) out[(size_t)(ti.row0 + c0 + j) * p.ld_routed + col] = __uint_as_float(v[j]);
+          } else if (routed) {
             uint16_t* out = static_cast<uint16_t*>(p.out_routed);
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
@@ -393,15 +399,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r,
                     __bfloat16_as_ushort(__float2bfloat16_rn(h));
               }
             }
-            uint16_t* gs = routed ? p.g_routed : p.g_shared;
-            uint16_t* us = routed ? p.u_routed : p.u_shared;
+            float* gs = routed ? p.g_routed : p.g_shared;
+            float* us = routed ? p.u_routed : p.u_shared;
             if (gs != nullptr) {
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
                 if (j < nj) {
                   const size_t at = (size_t)(ti.row0 + c0 + j) * ld + col;
-                  gs[at] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
-                  us[at] = __bfloat16_as_ushort(__float2bfloat16_rn(up_buf[j * 64 + frow]));
+                  gs[at] = __uint_as_float(v[j]);
+                  us[at] = up_buf[j * 64 + frow];
                 }
               }
             }
@@ -557,6 +563,7 @@ cudaError_t launch_grouped_gemms(const Shape& s, const GroupedGemmArgs& a, int n
     p.a_evict_first = small ? 1 : 0;
     p.offsets = a.offsets;
     p.out_routed = a.y_perm;
+    p.routed_f32 = a.y_perm_f32 ? 1 : 0;
     p.ld_routed = s.d;
     p.out_shared = a.y_shared;
     p.ld_shared = s.d;

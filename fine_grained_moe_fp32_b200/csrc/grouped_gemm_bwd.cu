@@ -68,8 +68,9 @@ struct BwdParams {
   void* out_shared;
   int ld_shared;
   int shared_f32;
+  int out_f32;                             // wgrad: fp32 weight gradients (else bf16)
   int64_t gstride_routed, gstride_shared;  // wgrad: elements between groups' outputs
-  const uint16_t *g_routed, *u_routed, *g_shared, *u_shared;  // dgrad-down: pre-activations
+  const float *g_routed, *u_routed, *g_shared, *u_shared;  // dgrad-down: fp32 pre-activations
   int ld_gu_routed, ld_gu_shared;
   int ucol_routed, ucol_shared;  // dgrad-down: column of dU in the output
   unsigned int* status;
@@ -387,32 +388,26 @@ grouped_gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmA_r,
     int acc = 0;
     uint32_t acc_phase = 0;
     const int et = threadIdx.x - 64;  // 0..127 over the epilogue warps
-    // SwiGLU backward: this thread's share of the g / u rows of one 32-token
-    // chunk (4 x 16 bytes each), loaded a chunk ahead so the global latency
-    // overlaps the accumulator wait and the previous chunk's work
-    uint4 gpre[4], upre[4];
+    // SwiGLU backward: this thread's feature (its TMEM lane) of the fp32 g / u
+    // rows of one 32-token chunk.  For each token the warp's 32 lanes read 32
+    // consecutive features (128 coalesced bytes); the loads are issued before
+    // the accumulator is read so their latency overlaps it.
+    float gv[32], uv[32];
     auto load_gu = [&](const Tile& t, int c0) {
       const bool routed = t.g < p.E;
-      const uint16_t* gsrc = routed ? p.g_routed : p.g_shared;
-      const uint16_t* usrc = routed ? p.u_routed : p.u_shared;
+      const float* gsrc = routed ? p.g_routed : p.g_shared;
+      const float* usrc = routed ? p.u_routed : p.u_shared;
       const int ldgu = routed ? p.ld_gu_routed : p.ld_gu_shared;
       const int nj = min(32, t.nrows - c0);
+      const size_t at0 = (size_t)(t.row0 + c0) * ldgu + t.mt * 128 + mrow;
 #pragma unroll
-      for (int it = 0; it < 4; ++it) {
-        const int i = et + it * kEpiThreads;
-        const int r = i >> 4, cv = i & 15;
-        gpre[it] = make_uint4(0, 0, 0, 0);
-        upre[it] = gpre[it];
-        if (r < nj) {
-          const size_t at = (size_t)(t.row0 + c0 + r) * ldgu + t.mt * 128 + cv * 8;
-          gpre[it] = *reinterpret_cast<const uint4*>(gsrc + at);
-          upre[it] = *reinterpret_cast<const uint4*>(usrc + at);
-        }
+      for (int j = 0; j < 32; ++j) {
+        gv[j] = j < nj ? gsrc[at0 + (size_t)j * ldgu] : 0.f;
+        uv[j] = j < nj ? usrc[at0 + (size_t)j * ldgu] : 0.f;
       }
     };
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       const Tile t = decode<MODE>(ctl, p, tile);
-      if (MODE == kDgradDown) load_gu(t, 0);
       bool bad = aborted(ctl);
       if (!bad && !mbar_wait_bounded(smem_u32(&ctl.tfull[acc]), acc_phase, p.wait_limit_ns)) {
         record_timeout(ctl, p);
@@ -424,59 +419,66 @@ grouped_gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmA_r,
       const uint32_t tbase = tmem_base + (uint32_t)(acc * kNT) + ((uint32_t)(q * 32) << 16);
       const int ncols = MODE == kWgrad ? t.n : t.nrows;
       for (int c0 = 0; c0 < ncols; c0 += 32) {
+        if (MODE == kDgradDown) load_gu(t, c0);
         uint32_t v[32];
         tmem_ld_32x32b_x32(tbase + (uint32_t)c0, v);
         tmem_ld_wait();
         const int nj = min(32, ncols - c0);
         if (MODE == kWgrad) {
-          // dW[group][mt*128 + mrow][ncol0 + c0 + j], bf16, 16-byte stores
+          // dW[group][mt*128 + mrow][ncol0 + c0 + j], 16-byte stores of bf16
+          // (8 values) or fp32 (4 values)
           const bool second = p.m_split > 0 && t.mt >= p.m_split;
           const int mt = second ? t.mt - p.m_split : t.mt;
-          uint16_t* out = static_cast<uint16_t*>(
-              second ? (routed ? p.out2_routed : p.out2_shared)
-                     : (routed ? p.out_routed : p.out_shared));
+          void* out = second ? (routed ? p.out2_routed : p.out2_shared)
+                             : (routed ? p.out_routed : p.out_shared);
           const int ldo = routed ? p.ntot_routed : p.ntot_shared;
           const int64_t gbase = routed ? (int64_t)t.g * p.gstride_routed
                                        : (int64_t)(t.g - p.E) * p.gstride_shared;
-          uint16_t* dst = out + gbase + (int64_t)(mt * 128 + mrow) * ldo + t.ncol0 + c0;
+          const int64_t at = gbase + (int64_t)(mt * 128 + mrow) * ldo + t.ncol0 + c0;
           const bool zero = t.kchunks == 0;  // no tokens: the gradient is zero
+          if (p.out_f32) {
+            float* dst = static_cast<float*>(out) + at;
 #pragma unroll
-          for (int j8 = 0; j8 < 4; ++j8) {
-            if (j8 * 8 < nj) {
-              uint32_t w[4];
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float lo = zero ? 0.f : __uint_as_float(v[j8 * 8 + 2 * i]);
-                const float hi = zero ? 0.f : __uint_as_float(v[j8 * 8 + 2 * i + 1]);
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);  // one paired cvt
-                w[i] = *reinterpret_cast<const uint32_t*>(&h2);
+            for (int j4 = 0; j4 < 8; ++j4) {
+              if (j4 * 4 < nj) {
+                const uint4 w = zero ? make_uint4(0, 0, 0, 0)
+                                     : make_uint4(v[j4 * 4], v[j4 * 4 + 1], v[j4 * 4 + 2],
+                                                  v[j4 * 4 + 3]);
+                *reinterpret_cast<uint4*>(dst + j4 * 4) = w;
               }
-              *reinterpret_cast<uint4*>(dst + j8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          } else {
+            uint16_t* dst = static_cast<uint16_t*>(out) + at;
+#pragma unroll
+            for (int j8 = 0; j8 < 4; ++j8) {
+              if (j8 * 8 < nj) {
+                uint32_t w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const float lo = zero ? 0.f : __uint_as_float(v[j8 * 8 + 2 * i]);
+                  const float hi = zero ? 0.f : __uint_as_float(v[j8 * 8 + 2 * i + 1]);
+                  const __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);  // one paired cvt
+                  w[i] = *reinterpret_cast<const uint32_t*>(&h2);
+                }
+                *reinterpret_cast<uint4*>(dst + j8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+              }
             }
           }
         } else if (MODE == kDgradDown) {
-          // SwiGLU backward on a 32-token x 128-feature tile staged in smem:
-          // g and u come in, and dG / dU go out, as coalesced 16-byte rows;
-          // each thread then works on its own feature (TMEM lane) in place.
+          // SwiGLU backward: each thread works on its own feature (TMEM lane)
+          // from the fp32 g and u in registers; dG / dU are staged in smem as
+          // a 32-token x 128-feature bf16 tile and go out as coalesced
+          // 16-byte rows.
           const int f0 = t.mt * 128;
           uint16_t* out = static_cast<uint16_t*>(routed ? p.out_routed : p.out_shared);
           const int ldo = routed ? p.ld_routed : p.ld_shared;
           const int ucol = routed ? p.ucol_routed : p.ucol_shared;
 #pragma unroll
-          for (int it = 0; it < 4; ++it) {
-            const int i = et + it * kEpiThreads;
-            const int r = i >> 4, cv = i & 15;
-            *reinterpret_cast<uint4*>(epi_g + r * 128 + cv * 8) = gpre[it];
-            *reinterpret_cast<uint4*>(epi_u + r * 128 + cv * 8) = upre[it];
-          }
-          named_bar_sync(1, kEpiThreads);
-          if (c0 + 32 < ncols) load_gu(t, c0 + 32);  // next chunk, in flight meanwhile
-#pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (j < nj) {
               const float dh = __uint_as_float(v[j]);
-              const float g = __uint_as_float((uint32_t)epi_g[j * 128 + mrow] << 16);
-              const float u = __uint_as_float((uint32_t)epi_u[j * 128 + mrow] << 16);
+              const float g = gv[j];
+              const float u = uv[j];
               const float sg = sigmoid_f(g);
               const float dg = dh * u * (sg * (1.0f + g * (1.0f - sg)));
               const float du = dh * (g * sg);
@@ -595,7 +597,7 @@ cudaError_t launch_backward_gemms(const Shape& s, const BackwardGemmArgs& a, int
   CUtensorMap m[6];
   cudaError_t err;
   if (s.S > 0 && s.T == 0) {  // no tokens: the shared experts' gradients are zero
-    const size_t bytes = (size_t)s.S * s.I * s.d * 2;
+    const size_t bytes = (size_t)s.S * s.I * s.d * (a.dw_f32 ? 4 : 2);
     if ((err = cudaMemsetAsync(a.dws1, 0, bytes, st)) != cudaSuccess ||
         (err = cudaMemsetAsync(a.dws3, 0, bytes, st)) != cudaSuccess ||
         (err = cudaMemsetAsync(a.dws2, 0, bytes, st)) != cudaSuccess)
@@ -660,6 +662,7 @@ cudaError_t launch_backward_gemms(const Shape& s, const BackwardGemmArgs& a, int
     p.b_step_shared = s.I;
     p.out_routed = a.dw2;
     p.out_shared = a.dws2;
+    p.out_f32 = a.dw_f32 ? 1 : 0;
     p.gstride_routed = p.gstride_shared = (int64_t)s.d * s.I;
     if ((err = launch_bwd<kWgrad>(m, p, num_sms, st)) != cudaSuccess) return err;
     if ((err = mark(1)) != cudaSuccess) return err;
@@ -723,6 +726,7 @@ cudaError_t launch_backward_gemms(const Shape& s, const BackwardGemmArgs& a, int
     p.out2_routed = a.dw3;
     p.out_shared = a.dws1;
     p.out2_shared = a.dws3;
+    p.out_f32 = a.dw_f32 ? 1 : 0;
     p.gstride_routed = p.gstride_shared = (int64_t)s.I * s.d;
     if ((err = launch_bwd<kWgrad>(m, p, num_sms, st)) != cudaSuccess) return err;
   }

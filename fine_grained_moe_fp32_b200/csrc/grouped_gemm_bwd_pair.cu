@@ -83,7 +83,8 @@ struct PBParams {
   int b_c0_routed, b_c0_shared, b_step_shared;  // wgrad B columns
   void *out_routed, *out_shared;  // dgrads (the weight gradients go through TMA store maps)
   int ld_routed, ld_shared;
-  const uint16_t *g_routed, *u_routed, *g_shared, *u_shared;  // dgrad-down pre-activations
+  int out_f32;                    // wgrad: the store maps are fp32 (else bf16)
+  const float *g_routed, *u_routed, *g_shared, *u_shared;  // dgrad-down fp32 pre-activations
   int ld_gu_routed, ld_gu_shared;
   int ucol_routed, ucol_shared;  // dgrad-down: column of dU in the output
   unsigned int* status;
@@ -208,9 +209,10 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
   extern __shared__ uint8_t dsmem_raw[];
   const uint32_t raw = smem_u32(dsmem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
-  // epilogue staging, 32 KB: per dH epilogue group the SwiGLU backward's g
-  // then u tiles ([32][128] bf16 each), or per weight-gradient epilogue warp
-  // one 4 KB store buffer (32 rows x 64 columns of bf16, 128-byte swizzle)
+  // epilogue staging, 32 KB: per dH epilogue group the SwiGLU backward's dG
+  // then dU tiles ([32][128] bf16 each), or per weight-gradient epilogue warp
+  // one 4 KB store buffer (32 rows x 64 columns of bf16 or 32 x 32 of fp32,
+  // 128-byte swizzle)
   uint8_t* epi = dsmem_raw + (sbase - raw) + STAGES * kStageBytes;
   uint16_t* epi_g = reinterpret_cast<uint16_t*>(epi);
 
@@ -478,26 +480,22 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
     const int gbar = 1 + 2 * grp;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&ctl.tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&ctl.tempty[1]), 0);
-    // SwiGLU backward: this thread's share of the g / u rows of one 32-token
-    // chunk, loaded a chunk ahead of its use
-    uint4 gpre[4], upre[4];
+    // SwiGLU backward: this thread's feature (its TMEM lane) of the fp32 g / u
+    // rows of one 32-token chunk.  For each token the warp's 32 lanes read 32
+    // consecutive features (128 coalesced bytes); the loads are issued before
+    // the accumulator is read so their latency overlaps it.
+    float gv[32], uv[32];
     auto load_gu = [&](const PBTile& t, int f0, int c0) {
       const bool routed = t.g < p.E;
-      const uint16_t* gsrc = routed ? p.g_routed : p.g_shared;
-      const uint16_t* usrc = routed ? p.u_routed : p.u_shared;
+      const float* gsrc = routed ? p.g_routed : p.g_shared;
+      const float* usrc = routed ? p.u_routed : p.u_shared;
       const int ldgu = routed ? p.ld_gu_routed : p.ld_gu_shared;
       const int nj = min(32, t.nrows - c0);
+      const size_t at0 = (size_t)(t.row0 + c0) * ldgu + f0 + mrow;
 #pragma unroll
-      for (int it = 0; it < 4; ++it) {
-        const int i = eg + it * kGrpThreads;
-        const int r = i >> 4, cv = i & 15;
-        gpre[it] = make_uint4(0, 0, 0, 0);
-        upre[it] = gpre[it];
-        if (r < nj) {
-          const size_t at = (size_t)(t.row0 + c0 + r) * ldgu + f0 + cv * 8;
-          gpre[it] = *reinterpret_cast<const uint4*>(gsrc + at);
-          upre[it] = *reinterpret_cast<const uint4*>(usrc + at);
-        }
+      for (int j = 0; j < 32; ++j) {
+        gv[j] = j < nj ? gsrc[at0 + (size_t)j * ldgu] : 0.f;
+        uv[j] = j < nj ? usrc[at0 + (size_t)j * ldgu] : 0.f;
       }
     };
     int acc = 0;
@@ -522,7 +520,6 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
       const int r0 = t.mt * 256 + (int)rank * 128;
       // rows past the group's M extent hold zero-filled products: skipped
       const bool live = r0 < (routed ? p.mext_routed : p.mext_shared);
-      if (MODE == kPDgradDown && live) load_gu(t, r0, grp * 32);
       bool bad = pb_aborted(ctl);
       if (!bad && !mbar_wait_bounded(smem_u32(&ctl.tfull[acc]), acc_phase, p.wait_limit_ns)) {
         pb_timeout(ctl, p);
@@ -559,6 +556,40 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
         constexpr int kStep = 64 * (kEpiWarps / 4);
         const int cfirst = 64 * (ew >> 2);
         uint32_t va[32], vb[32];
+        if (p.out_f32) {
+          // fp32: each 32-column half is one 32 x 32 box (128-byte rows),
+          // staged in this warp's buffer after the previous store has read it
+          auto put = [&](const uint32_t (&v)[32], int col) {
+            uint8_t* buf = epi + ew * (kBufs * 4096) + (nstore % kBufs) * 4096u;
+            if (lane == 0) bulk_wait_group_read<kBufs - 1>();
+            __syncwarp();
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {  // 128-byte swizzle: 16-byte chunk c ^ (row % 8)
+              const int phys = c ^ (lane & 7);
+              *reinterpret_cast<uint4*>(buf + lane * 128 + phys * 16) =
+                  zero ? make_uint4(0, 0, 0, 0)
+                       : make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(tO, smem_u32(buf), t.ncol0 + col, orow, plane);
+              bulk_commit_group();
+            }
+            ++nstore;
+          };
+          for (int c0 = cfirst; c0 < ncols; c0 += kStep) {
+            tmem_ld_32x32b_x32(tbase + (uint32_t)c0, va);
+            tmem_ld_32x32b_x32(tbase + (uint32_t)(c0 + 32), vb);
+            tmem_ld_wait();
+            if (c0 + kStep >= ncols) {  // this warp's last columns are in registers
+              release(acc);
+              freed = true;
+            }
+            put(va, c0);
+            put(vb, c0 + 32);
+          }
+        } else {
         if (cfirst < ncols) {
           tmem_ld_32x32b_x32(tbase + (uint32_t)cfirst, va);
           tmem_ld_32x32b_x32(tbase + (uint32_t)(cfirst + 32), vb);
@@ -603,8 +634,10 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
             }
           }
         }
+        }
       }
       for (int c0 = grp * 32; MODE != kPWgrad && live && c0 < ncols; c0 += kChunkStep) {
+        if (MODE == kPDgradDown) load_gu(t, r0, c0);
         uint32_t v[32];
         tmem_ld_32x32b_x32(tbase + (uint32_t)c0, v);
         tmem_ld_wait();
@@ -615,21 +648,11 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
           const int ldo = routed ? p.ld_routed : p.ld_shared;
           const int ucol = routed ? p.ucol_routed : p.ucol_shared;
 #pragma unroll
-          for (int it = 0; it < 4; ++it) {
-            const int i = eg + it * kGrpThreads;
-            const int r = i >> 4, cv = i & 15;
-            *reinterpret_cast<uint4*>(gbuf + r * 128 + cv * 8) = gpre[it];
-            *reinterpret_cast<uint4*>(ubuf + r * 128 + cv * 8) = upre[it];
-          }
-          named_bar_sync(gbar, kGrpThreads);
-          // this group's next chunk, in flight meanwhile
-          if (c0 + kChunkStep < ncols) load_gu(t, r0, c0 + kChunkStep);
-#pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (j < nj) {
               const float dh = __uint_as_float(v[j]);
-              const float g = __uint_as_float((uint32_t)gbuf[j * 128 + mrow] << 16);
-              const float u = __uint_as_float((uint32_t)ubuf[j * 128 + mrow] << 16);
+              const float g = gv[j];
+              const float u = uv[j];
               const float sg = pb_sigmoid(g);
               const float dg = dh * u * (sg * (1.0f + g * (1.0f - sg)));
               const float du = dh * (g * sg);
@@ -704,17 +727,20 @@ bool make_map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 output (inner, rows, planes) written by TMA stores of 64 x 32 boxes,
-// 128-byte swizzle (the staging layout of the weight-gradient epilogue).
-bool make_store_map3(CUtensorMap* m, void* base, uint64_t inner, uint64_t rows, uint64_t planes) {
+// Output (inner, rows, planes) written by TMA stores of 128-byte x 32-row
+// boxes with the 128-byte swizzle (the staging layout of the weight-gradient
+// epilogue): 64 columns of bf16, or 32 columns of fp32 when f32.
+bool make_store_map3(CUtensorMap* m, void* base, uint64_t inner, uint64_t rows, uint64_t planes,
+                     bool f32) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
+  const uint64_t es = f32 ? 4 : 2;
   cuuint64_t dims[3] = {inner, rows, planes};
-  cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
-  cuuint32_t box[3] = {64u, 32u, 1u};
+  cuuint64_t strides[2] = {inner * es, inner * rows * es};
+  cuuint32_t box[3] = {f32 ? 32u : 64u, 32u, 1u};
   cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base,
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -827,8 +853,8 @@ cudaError_t launch_backward_gemms_pair(const Shape& s, const BackwardGemmArgs& a
     else
       m[3] = m[0], m[5] = m[2];
     m[4] = m[3];
-    ok = ok && make_store_map3(&m[6], a.dw2, s.I, s.d, s.E);
-    if (shared) ok = ok && make_store_map3(&m[8], a.dws2, s.I, s.d, s.S);
+    ok = ok && make_store_map3(&m[6], a.dw2, s.I, s.d, s.E, a.dw_f32);
+    if (shared) ok = ok && make_store_map3(&m[8], a.dws2, s.I, s.d, s.S, a.dw_f32);
     else m[8] = m[6];
     m[7] = m[6];
     m[9] = m[8];
@@ -840,6 +866,7 @@ cudaError_t launch_backward_gemms_pair(const Shape& s, const BackwardGemmArgs& a
     p.ntot_routed = p.ntot_shared = s.I;
     p.nt_routed = p.nt_shared = (int)ceil_div(s.I, kNT);
     p.b_step_shared = s.I;
+    p.out_f32 = a.dw_f32 ? 1 : 0;
     if ((err = launch_pb<kPWgrad, kWgradKSubs, kWgradStages>(m, p, num_sms, st)) != cudaSuccess) return err;
     if ((err = mark(1)) != cudaSuccess) return err;
   }
@@ -882,11 +909,11 @@ cudaError_t launch_backward_gemms_pair(const Shape& s, const BackwardGemmArgs& a
     else
       m[3] = m[0], m[5] = m[2];
     m[4] = m[3];
-    ok = ok && make_store_map3(&m[6], a.dw1, s.d, s.I, s.E) &&
-         make_store_map3(&m[7], a.dw3, s.d, s.I, s.E);
+    ok = ok && make_store_map3(&m[6], a.dw1, s.d, s.I, s.E, a.dw_f32) &&
+         make_store_map3(&m[7], a.dw3, s.d, s.I, s.E, a.dw_f32);
     if (shared)
-      ok = ok && make_store_map3(&m[8], a.dws1, s.d, s.I, s.S) &&
-           make_store_map3(&m[9], a.dws3, s.d, s.I, s.S);
+      ok = ok && make_store_map3(&m[8], a.dws1, s.d, s.I, s.S, a.dw_f32) &&
+           make_store_map3(&m[9], a.dws3, s.d, s.I, s.S, a.dw_f32);
     else
       m[8] = m[6], m[9] = m[7];
     if (!ok) return cudaErrorInvalidValue;
@@ -902,6 +929,7 @@ cudaError_t launch_backward_gemms_pair(const Shape& s, const BackwardGemmArgs& a
     p.a_step_shared = s.I;
     p.ntot_routed = p.ntot_shared = s.d;
     p.nt_routed = p.nt_shared = (int)ceil_div(s.d, kNT);
+    p.out_f32 = a.dw_f32 ? 1 : 0;
     if ((err = launch_pb<kPWgrad, kWgradKSubs, kWgradStages>(m, p, num_sms, st)) != cudaSuccess) return err;
   }
   return mark(3);

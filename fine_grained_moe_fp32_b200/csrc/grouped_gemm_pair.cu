@@ -64,7 +64,8 @@ struct PairParams {
   void* out_shared;
   int ld_shared;
   int shared_f32;
-  uint16_t *g_routed, *u_routed, *g_shared, *u_shared;
+  int routed_f32;  // down GEMM: routed rows stored in fp32 (else bf16)
+  float *g_routed, *u_routed, *g_shared, *u_shared;  // training: fp32 pre-activations
   unsigned int* status;
   uint64_t wait_limit_ns;
 };
@@ -369,7 +370,12 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
         const int nj = min(32, t.nrows - c0);
         if (MODE == kPairDown) {
           const int col = t.ft * 256 + (int)rank * 128 + frow;
-          if (routed) {
+          if (routed && p.routed_f32) {
+            float* out = static_cast<float*>(p.out_routed);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nj) out[(size_t)(t.row0 + c0 + j) * p.ld_routed + col] = __uint_as_float(v[j]);
+          } else if (routed) {
             uint16_t* out = static_cast<uint16_t*>(p.out_routed);
 #pragma unroll
             for (int j = 0; j < 32; ++j)
@@ -412,16 +418,16 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
                   __bfloat16_as_ushort(__float2bfloat16_rn(h));
             }
           }
-          uint16_t* gs = routed ? p.g_routed : p.g_shared;
-          uint16_t* us = routed ? p.u_routed : p.u_shared;
+          float* gs = routed ? p.g_routed : p.g_shared;
+          float* us = routed ? p.u_routed : p.u_shared;
           if (gs != nullptr) {
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) {
               const int j = jb + jj;
               if (j < nj) {
                 const size_t at = (size_t)(t.row0 + c0 + j) * ld + col;
-                gs[at] = __bfloat16_as_ushort(__float2bfloat16_rn(gate_buf[j * 64 + f]));
-                us[at] = __bfloat16_as_ushort(__float2bfloat16_rn(up_buf[j * 64 + f]));
+                gs[at] = gate_buf[j * 64 + f];
+                us[at] = up_buf[j * 64 + f];
               }
             }
           }
@@ -582,6 +588,7 @@ cudaError_t launch_grouped_gemms_pair(const Shape& s, const GroupedGemmArgs& a, 
     p.a_rows_group = s.d;
     p.offsets = a.offsets;
     p.out_routed = a.y_perm;
+    p.routed_f32 = a.y_perm_f32 ? 1 : 0;
     p.ld_routed = s.d;
     p.out_shared = a.y_shared;
     p.ld_shared = s.d;

@@ -97,7 +97,7 @@ moe_ws_layout make_layout(const Shape& s) {
   L.permute_scratch = take(permute_scratch_bytes(s));
   L.x_perm = take((size_t)s.cap * s.d * 2);
   L.h_perm = take((size_t)s.cap * s.I * 2);
-  L.y_perm = take((size_t)s.cap * s.d * 2);
+  L.y_perm = take((size_t)s.cap * s.d * 4);
   L.h_shared = take((size_t)s.T * s.S * s.I * 2);
   L.y_shared = take((size_t)s.T * s.d * 4);
   L.total = off;
@@ -114,10 +114,10 @@ moe_train_layout make_train_layout(const Shape& s) {
     return at;
   };
   const size_t SI = (size_t)s.S * s.I;
-  L.g_perm = take((size_t)s.cap * s.I * 2);
-  L.u_perm = take((size_t)s.cap * s.I * 2);
-  L.g_shared = take((size_t)s.T * SI * 2);
-  L.u_shared = take((size_t)s.T * SI * 2);
+  L.g_perm = take((size_t)s.cap * s.I * 4);
+  L.u_perm = take((size_t)s.cap * s.I * 4);
+  L.g_shared = take((size_t)s.T * SI * 4);
+  L.u_shared = take((size_t)s.T * SI * 4);
   L.dy_perm = take((size_t)s.cap * s.d * 2);
   L.dw = take((size_t)s.T * s.k * 4);
   L.dz = take((size_t)s.T * s.E * 4);
@@ -215,7 +215,7 @@ int moe_permute(const moe_dims* dims, const int32_t* topk_idx, const moe_bf16* x
 
 int moe_grouped_swiglu(const moe_dims* dims, const moe_bf16* x_perm, const int32_t* offsets,
                        const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
-                       moe_bf16* h_perm, moe_bf16* y_perm, void* stream) {
+                       moe_bf16* h_perm, float* y_perm, void* stream) {
   Shape s;
   int rc = check_dims(dims, &s);
   if (rc != MOE_OK) return rc;
@@ -239,7 +239,7 @@ int moe_grouped_swiglu(const moe_dims* dims, const moe_bf16* x_perm, const int32
                                           static_cast<cudaStream_t>(stream)));
 }
 
-int moe_combine(const moe_dims* dims, const moe_bf16* y_perm, const int32_t* row_of,
+int moe_combine(const moe_dims* dims, const float* y_perm, const int32_t* row_of,
                 const float* topk_w, const float* y_shared, moe_bf16* y, void* stream) {
   Shape s;
   int rc = check_dims(dims, &s);
@@ -307,7 +307,7 @@ int forward_impl(const moe_dims* dims, const moe_bf16* x, const float* w_gate, c
   int32_t* tor = at<int32_t>(ws, L.token_of_row);
   uint16_t* x_perm = at<uint16_t>(ws, L.x_perm);
   uint16_t* h_perm = at<uint16_t>(ws, L.h_perm);
-  uint16_t* y_perm = at<uint16_t>(ws, L.y_perm);
+  float* y_perm = at<float>(ws, L.y_perm);
   uint16_t* h_sh = at<uint16_t>(ws, L.h_shared);
   float* y_sh = at<float>(ws, L.y_shared);
 
@@ -338,10 +338,10 @@ int forward_impl(const moe_dims* dims, const moe_bf16* x, const float* w_gate, c
     a.y_shared = y_sh;
   }
   if (train) {
-    a.g_perm = at<uint16_t>(ws, TL.g_perm);
-    a.u_perm = at<uint16_t>(ws, TL.u_perm);
-    a.g_shared = at<uint16_t>(ws, TL.g_shared);
-    a.u_shared = at<uint16_t>(ws, TL.u_shared);
+    a.g_perm = at<float>(ws, TL.g_perm);
+    a.u_perm = at<float>(ws, TL.u_perm);
+    a.g_shared = at<float>(ws, TL.g_shared);
+    a.u_shared = at<float>(ws, TL.u_shared);
   }
   e = launch_grouped_gemms(s, a, di->num_sms, di->status, g_wait_limit_ns, st,
                            g_phase_on ? g_phase_events[3] : nullptr);
@@ -393,11 +393,18 @@ int moe_forward_train(const moe_dims* dims, const moe_bf16* x, const float* w_ga
                       workspace_bytes, stream, true);
 }
 
-int moe_backward(const moe_dims* dims, const moe_bf16* x, const float* w_gate, const moe_bf16* w1,
-                 const moe_bf16* w3, const moe_bf16* w2, const moe_bf16* ws1, const moe_bf16* ws3,
-                 const moe_bf16* ws2, const moe_bf16* dy, void* workspace, size_t workspace_bytes,
-                 moe_bf16* dx, float* dw_gate, moe_bf16* dw1, moe_bf16* dw3, moe_bf16* dw2,
-                 moe_bf16* dws1, moe_bf16* dws3, moe_bf16* dws2, void* stream) {
+}  // extern "C"
+
+namespace moe {
+namespace {
+
+// The backward; `f32` selects fp32 dx and weight gradients (else bf16).
+int backward_impl(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
+                  const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
+                  const moe_bf16* ws1, const moe_bf16* ws3, const moe_bf16* ws2,
+                  const moe_bf16* dy, void* workspace, size_t workspace_bytes, void* dx,
+                  float* dw_gate, void* dw1, void* dw3, void* dw2, void* dws1, void* dws3,
+                  void* dws2, void* stream, bool f32) {
   Shape s;
   int rc = check_dims(dims, &s);
   if (rc != MOE_OK) return rc;
@@ -425,7 +432,7 @@ int moe_backward(const moe_dims* dims, const moe_bf16* x, const float* w_gate, c
   BackwardMiscArgs m{};
   m.x = x;
   m.dy = dy;
-  m.y_perm = at<uint16_t>(ws, L.y_perm);
+  m.y_perm = at<float>(ws, L.y_perm);
   m.w_gate = w_gate;
   m.probs = at<float>(ws, L.probs);
   m.topk_w = at<float>(ws, L.topk_w);
@@ -442,6 +449,7 @@ int moe_backward(const moe_dims* dims, const moe_bf16* x, const float* w_gate, c
   m.dwg_partials = at<float>(ws, TL.dwg_partials);
   m.dw_gate = dw_gate;
   m.dx = dx;
+  m.dx_f32 = f32;
   cudaError_t e = bwd_phase(0, st);
   if (e == cudaSuccess) e = launch_backward_misc_pre(s, m, st);
   if (e == cudaSuccess) e = bwd_phase(1, st);
@@ -459,10 +467,10 @@ int moe_backward(const moe_dims* dims, const moe_bf16* x, const float* w_gate, c
   g.x_perm = at<uint16_t>(ws, L.x_perm);
   g.h_perm = at<uint16_t>(ws, L.h_perm);
   g.h_shared = at<uint16_t>(ws, L.h_shared);
-  g.g_perm = at<uint16_t>(ws, TL.g_perm);
-  g.u_perm = at<uint16_t>(ws, TL.u_perm);
-  g.g_shared = at<uint16_t>(ws, TL.g_shared);
-  g.u_shared = at<uint16_t>(ws, TL.u_shared);
+  g.g_perm = at<float>(ws, TL.g_perm);
+  g.u_perm = at<float>(ws, TL.u_perm);
+  g.g_shared = at<float>(ws, TL.g_shared);
+  g.u_shared = at<float>(ws, TL.u_shared);
   g.dy = dy;
   g.dy_perm = m.dy_perm;
   g.dgu_perm = at<uint16_t>(ws, TL.dgu_perm);
@@ -475,12 +483,39 @@ int moe_backward(const moe_dims* dims, const moe_bf16* x, const float* w_gate, c
   g.dws1 = dws1;
   g.dws3 = dws3;
   g.dws2 = dws2;
+  g.dw_f32 = f32;
   e = launch_backward_gemms(s, g, di->num_sms, di->status, g_wait_limit_ns, st,
                             g_bwd_phase_on ? &g_phase_events[kFwdEvents + 2] : nullptr);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   e = launch_backward_misc_post(s, m, st);
   if (e == cudaSuccess) e = bwd_phase(6, st);
   return cuda_status(e);
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+int moe_backward(const moe_dims* dims, const moe_bf16* x, const float* w_gate, const moe_bf16* w1,
+                 const moe_bf16* w3, const moe_bf16* w2, const moe_bf16* ws1, const moe_bf16* ws3,
+                 const moe_bf16* ws2, const moe_bf16* dy, void* workspace, size_t workspace_bytes,
+                 moe_bf16* dx, float* dw_gate, moe_bf16* dw1, moe_bf16* dw3, moe_bf16* dw2,
+                 moe_bf16* dws1, moe_bf16* dws3, moe_bf16* dws2, void* stream) {
+  return backward_impl(dims, x, w_gate, w1, w3, w2, ws1, ws3, ws2, dy, workspace,
+                       workspace_bytes, dx, dw_gate, dw1, dw3, dw2, dws1, dws3, dws2, stream,
+                       false);
+}
+
+int moe_backward_f32(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
+                     const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
+                     const moe_bf16* ws1, const moe_bf16* ws3, const moe_bf16* ws2,
+                     const moe_bf16* dy, void* workspace, size_t workspace_bytes, float* dx,
+                     float* dw_gate, float* dw1, float* dw3, float* dw2, float* dws1,
+                     float* dws3, float* dws2, void* stream) {
+  return backward_impl(dims, x, w_gate, w1, w3, w2, ws1, ws3, ws2, dy, workspace,
+                       workspace_bytes, dx, dw_gate, dw1, dw3, dw2, dws1, dws3, dws2, stream,
+                       true);
 }
 
 }  // extern "C"
@@ -547,6 +582,7 @@ int moe_dense_swiglu(const moe_dims* dims, const moe_bf16* x, const moe_bf16* w1
   a.w2 = w2;
   a.h_perm = at<uint16_t>(workspace, dense_h_offset());
   a.y_perm = y;
+  a.y_perm_f32 = false;  // the dense FFN's output is the caller's bf16 y
   return cuda_status(
       launch_grouped_gemms(s, a, di->num_sms, di->status, g_wait_limit_ns, st, nullptr));
 }
@@ -715,7 +751,7 @@ int moe_ep_dispatch(const moe_dims* dims, int world, int rank, const moe_bf16* x
 int moe_ep_experts(const moe_dims* dims, int world, const moe_bf16* x, const moe_bf16* x_recv,
                    const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
                    const moe_bf16* ws1, const moe_bf16* ws3, const moe_bf16* ws2,
-                   moe_bf16* y_recv, void* workspace, size_t workspace_bytes, void* stream) {
+                   float* y_recv, void* workspace, size_t workspace_bytes, void* stream) {
   Shape s;
   int64_t rcap;
   moe_ep_layout L;
@@ -754,7 +790,7 @@ int moe_ep_experts(const moe_dims* dims, int world, const moe_bf16* x, const moe
                                           static_cast<cudaStream_t>(stream)));
 }
 
-int moe_ep_combine(const moe_dims* dims, int world, const moe_bf16* const* y_recv, moe_bf16* y,
+int moe_ep_combine(const moe_dims* dims, int world, const float* const* y_recv, moe_bf16* y,
                    void* workspace, size_t workspace_bytes, void* stream) {
   Shape s;
   int64_t rcap;

@@ -48,17 +48,18 @@ struct GroupedGemmArgs {
   const int32_t* offsets;  // [E+1]
   const uint16_t *w1, *w3, *w2;
   uint16_t* h_perm;  // [cap, I]
-  uint16_t* y_perm;  // [cap, d]
+  void* y_perm;      // [cap, d] fp32, or bf16 when !y_perm_f32 (the dense FFN's y)
+  bool y_perm_f32 = true;
   // shared experts (S > 0 and all non-null to enable)
   const uint16_t* x;  // [T, d]
   const uint16_t *ws1, *ws3, *ws2;
   uint16_t* h_shared;  // [T, S*I]
   float* y_shared;     // [T, d]
-  // training: pre-activations of the gate/up GEMM (null = not stored)
-  uint16_t* g_perm = nullptr;    // [cap, I]
-  uint16_t* u_perm = nullptr;    // [cap, I]
-  uint16_t* g_shared = nullptr;  // [T, S*I]
-  uint16_t* u_shared = nullptr;  // [T, S*I]
+  // training: pre-activations of the gate/up GEMM, fp32 (null = not stored)
+  float* g_perm = nullptr;    // [cap, I]
+  float* u_perm = nullptr;    // [cap, I]
+  float* g_shared = nullptr;  // [T, S*I]
+  float* u_shared = nullptr;  // [T, S*I]
 };
 // `between` (may be null) is recorded on `st` after the gate/up GEMM is launched.
 cudaError_t launch_grouped_gemms(const Shape& s, const GroupedGemmArgs& a, int num_sms,
@@ -77,13 +78,14 @@ struct BackwardGemmArgs {
   const uint16_t *w1, *w3, *w2, *ws1, *ws3, *ws2;
   const uint16_t *x, *x_perm;                             // forward inputs
   const uint16_t *h_perm, *h_shared;                      // forward activations
-  const uint16_t *g_perm, *u_perm, *g_shared, *u_shared;  // saved pre-activations
+  const float *g_perm, *u_perm, *g_shared, *u_shared;     // saved pre-activations (fp32)
   const uint16_t *dy, *dy_perm;  // upstream gradient: per token, and w * dy per segment row
   uint16_t* dgu_perm;    // [cap, 2I]  [dG | dU]
   uint16_t* dgu_shared;  // [T, 2*S*I]
   float* dx_perm;        // [cap, d]
   float* dx_shared;      // [T, d]
-  uint16_t *dw1, *dw3, *dw2, *dws1, *dws3, *dws2;
+  void *dw1, *dw3, *dw2, *dws1, *dws3, *dws2;  // bf16, or fp32 when dw_f32
+  bool dw_f32 = false;
 };
 // `events` (may be null): 4 events recorded after the dH/SwiGLU dgrad, the dW2
 // wgrad, the dX dgrad and the dW1/dW3 wgrads.
@@ -97,7 +99,8 @@ cudaError_t launch_backward_gemms(const Shape& s, const BackwardGemmArgs& a, int
 
 // ---- backward outside the expert GEMMs (backward.cu)
 struct BackwardMiscArgs {
-  const uint16_t *x, *dy, *y_perm;
+  const uint16_t *x, *dy;
+  const float* y_perm;  // [cap, d] routed expert outputs
   const float *w_gate, *probs, *topk_w;
   const int32_t *topk_idx, *row_of, *offsets, *token_of_row;
   uint16_t* dy_perm;    // [cap, d]
@@ -108,7 +111,8 @@ struct BackwardMiscArgs {
   float* dx_router;     // [T, d]
   float* dwg_partials;  // [splits, E, d]
   float* dw_gate;       // [E, d]
-  uint16_t* dx;         // [T, d]
+  void* dx;             // [T, d] bf16, or fp32 when dx_f32
+  bool dx_f32 = false;
 };
 int dwg_splits(const Shape& s);
 cudaError_t launch_backward_misc_pre(const Shape& s, const BackwardMiscArgs& a, cudaStream_t st);
@@ -123,13 +127,13 @@ cudaError_t launch_balance_stats(const Shape& s, int seq_len, const float* probs
 cudaError_t launch_bias_update(const Shape& s, const int32_t* counts, float gamma,
                                const float* bias_in, float* bias_out, cudaStream_t st);
 
-// ---- combine (combine.cu)
-cudaError_t launch_combine(const Shape& s, const uint16_t* y_perm, const int32_t* row_of,
+// ---- combine (combine.cu); routed expert outputs in fp32
+cudaError_t launch_combine(const Shape& s, const float* y_perm, const int32_t* row_of,
                            const float* topk_w, const float* y_shared, uint16_t* y,
                            cudaStream_t st);
 // expert parallel: rows pulled from the owners' receive buffers
 // y_recv[idx / (E/world)] at remote_row (rows < cap; -1 = skipped)
-cudaError_t launch_ep_combine(const Shape& s, int world, const uint16_t* const* y_recv,
+cudaError_t launch_ep_combine(const Shape& s, int world, const float* const* y_recv,
                               const int32_t* topk_idx, const int32_t* remote_row, int64_t cap,
                               const float* topk_w, const float* y_shared, uint16_t* y,
                               cudaStream_t st);

@@ -99,7 +99,7 @@ class EPGroup:
         self.views = M.ep_workspace_views(self.dm, self.world, self.ws)
         bf = dict(dtype=torch.bfloat16, device=self.device)
         self.x_recv = torch.empty((self.recv_cap, cfg.d), **bf)
-        self.y_recv = torch.empty((self.recv_cap, cfg.d), **bf)
+        self.y_recv = torch.empty((self.recv_cap, cfg.d), dtype=torch.float32, device=self.device)
         bufs = {"counts": self.views["counts"], "x_recv": self.x_recv, "y_recv": self.y_recv}
         local_h = {n: (*M.ipc_export(t), t.data_ptr()) for n, t in bufs.items()}
         addrs, self._opened = exchange_pointers(local_h, group)

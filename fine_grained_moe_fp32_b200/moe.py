@@ -28,6 +28,7 @@ EXPORTED = (
     "moe_workspace_size", "moe_forward_layout", "moe_forward", "moe_get_last_device_status",
     "moe_set_wait_limit_ns", "moe_set_phase_events", "moe_route_noalloc",
     "moe_train_workspace_size", "moe_train_layout_of", "moe_forward_train", "moe_backward",
+    "moe_backward_f32",
     "moe_balance_workspace_size", "moe_balance_stats", "moe_bias_update",
     "moe_dense_workspace_size", "moe_dense_swiglu",
     "moe_ep_recv_capacity", "moe_ep_workspace_size", "moe_ep_layout_of", "moe_ep_route",
@@ -101,6 +102,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_train_layout_of": (I, [P, ctypes.POINTER(MoeTrainLayout)]),
         "moe_forward_train": (I, [P, V, V, V, V, V, V, V, V, V, V, V, Z, V]),
         "moe_backward": (I, [P, V, V, V, V, V, V, V, V, V, V, Z, V, V, V, V, V, V, V, V, V]),
+        "moe_backward_f32": (I, [P, V, V, V, V, V, V, V, V, V, V, Z, V, V, V, V, V, V, V, V, V]),
         "moe_balance_workspace_size": (Z, [P, I]),
         "moe_balance_stats": (I, [P, I, V, V, ctypes.c_float, V, V, V, V, Z, V]),
         "moe_bias_update": (I, [P, V, ctypes.c_float, V, V, V]),
@@ -248,7 +250,7 @@ def grouped_swiglu(dm, x_perm, offsets, w1, w3, w2, h_perm, y_perm, stream=None)
     _expect(w3, torch.bfloat16, (dm.E, dm.I, dm.d), "w3")
     _expect(w2, torch.bfloat16, (dm.E, dm.d, dm.I), "w2")
     _expect(h_perm, torch.bfloat16, (cap, dm.I), "h_perm")
-    _expect(y_perm, torch.bfloat16, (cap, dm.d), "y_perm")
+    _expect(y_perm, torch.float32, (cap, dm.d), "y_perm")
     rc = load().moe_grouped_swiglu(ctypes.byref(dm), _ptr(x_perm), _ptr(offsets), _ptr(w1),
                                    _ptr(w3), _ptr(w2), _ptr(h_perm), _ptr(y_perm),
                                    _stream(stream))
@@ -257,7 +259,7 @@ def grouped_swiglu(dm, x_perm, offsets, w1, w3, w2, h_perm, y_perm, stream=None)
 
 def combine(dm, y_perm, row_of, topk_w, y_shared, y, stream=None):
     cap = capacity(dm)
-    _expect(y_perm, torch.bfloat16, (cap, dm.d), "y_perm")
+    _expect(y_perm, torch.float32, (cap, dm.d), "y_perm")
     _expect(row_of, torch.int32, (dm.T * dm.k,), "row_of")
     _expect(topk_w, torch.float32, (dm.T, dm.k), "topk_w")
     _expect(y_shared, torch.float32, (dm.T, dm.d), "y_shared")
@@ -307,20 +309,30 @@ def forward_train(dm, x, w_gate, bias, w1, w3, w2, ws1, ws3, ws2, y, workspace, 
 
 
 def backward(dm, x, w_gate, w1, w3, w2, ws1, ws3, ws2, dy, workspace, grads: dict, stream=None):
-    """grads: dict with preallocated dx, dw_gate, dw1, dw3, dw2, dws1, dws3, dws2."""
+    """grads: dict with preallocated dx, dw_gate, dw1, dw3, dw2, dws1, dws3, dws2.
+    dx and the expert weight gradients are all bf16 (moe_backward) or all fp32
+    (moe_backward_f32); dw_gate is fp32 either way."""
+    dt = grads["dw1"].dtype
+    if dt not in (torch.bfloat16, torch.float32):
+        raise TypeError(f"dw1: expected bf16 or fp32, got {dt}")
     _expect(dy, torch.bfloat16, (dm.T, dm.d), "dy")
-    _expect(grads["dx"], torch.bfloat16, (dm.T, dm.d), "dx")
+    _expect(grads["dx"], dt, (dm.T, dm.d), "dx")
     _expect(grads["dw_gate"], torch.float32, (dm.E, dm.d), "dw_gate")
-    _expect(grads["dw1"], torch.bfloat16, (dm.E, dm.I, dm.d), "dw1")
-    _expect(grads["dw3"], torch.bfloat16, (dm.E, dm.I, dm.d), "dw3")
-    _expect(grads["dw2"], torch.bfloat16, (dm.E, dm.d, dm.I), "dw2")
+    _expect(grads["dw1"], dt, (dm.E, dm.I, dm.d), "dw1")
+    _expect(grads["dw3"], dt, (dm.E, dm.I, dm.d), "dw3")
+    _expect(grads["dw2"], dt, (dm.E, dm.d, dm.I), "dw2")
+    for n, shape in (("dws1", (dm.n_shared, dm.I, dm.d)), ("dws3", (dm.n_shared, dm.I, dm.d)),
+                     ("dws2", (dm.n_shared, dm.d, dm.I))):
+        if grads.get(n) is not None:
+            _expect(grads[n], dt, shape, n)
     g = grads
-    rc = load().moe_backward(ctypes.byref(dm), _ptr(x), _ptr(w_gate), _ptr(w1), _ptr(w3),
-                             _ptr(w2), _ptr(ws1), _ptr(ws3), _ptr(ws2), _ptr(dy), _ptr(workspace),
-                             workspace.numel(), _ptr(g["dx"]), _ptr(g["dw_gate"]), _ptr(g["dw1"]),
-                             _ptr(g["dw3"]), _ptr(g["dw2"]), _ptr(g.get("dws1")),
-                             _ptr(g.get("dws3")), _ptr(g.get("dws2")), _stream(stream))
-    _check(rc, "moe_backward")
+    fn = load().moe_backward_f32 if dt == torch.float32 else load().moe_backward
+    rc = fn(ctypes.byref(dm), _ptr(x), _ptr(w_gate), _ptr(w1), _ptr(w3),
+            _ptr(w2), _ptr(ws1), _ptr(ws3), _ptr(ws2), _ptr(dy), _ptr(workspace),
+            workspace.numel(), _ptr(g["dx"]), _ptr(g["dw_gate"]), _ptr(g["dw1"]),
+            _ptr(g["dw3"]), _ptr(g["dw2"]), _ptr(g.get("dws1")),
+            _ptr(g.get("dws3")), _ptr(g.get("dws2")), _stream(stream))
+    _check(rc, "moe_backward_f32" if dt == torch.float32 else "moe_backward")
 
 
 def dense_dims(T, d, I) -> MoeDims:
@@ -416,7 +428,7 @@ def ep_dispatch(dm, world, rank, x, counts_of, x_recv, workspace, stream=None):
 def ep_experts(dm, world, x, x_recv, w1, w3, w2, ws1, ws3, ws2, y_recv, workspace, stream=None):
     El, rc = dm.E // world, ep_recv_capacity(dm, world)
     _expect(x_recv, torch.bfloat16, (rc, dm.d), "x_recv")
-    _expect(y_recv, torch.bfloat16, (rc, dm.d), "y_recv")
+    _expect(y_recv, torch.float32, (rc, dm.d), "y_recv")
     _expect(w1, torch.bfloat16, (El, dm.I, dm.d), "w1")
     _expect(w2, torch.bfloat16, (El, dm.d, dm.I), "w2")
     _check(load().moe_ep_experts(ctypes.byref(dm), int(world), _ptr(x), _ptr(x_recv), _ptr(w1),
@@ -509,7 +521,8 @@ class EPRanks:
         self.ws = [alloc_workspace(nbytes, self.device) for _ in range(world)]
         bf = dict(dtype=torch.bfloat16, device=self.device)
         self.x_recv = [torch.empty((self.recv_cap, cfg.d), **bf) for _ in range(world)]
-        self.y_recv = [torch.empty((self.recv_cap, cfg.d), **bf) for _ in range(world)]
+        self.y_recv = [torch.empty((self.recv_cap, cfg.d), dtype=torch.float32, device=self.device)
+                       for _ in range(world)]
         self.views = [ep_workspace_views(self.dm, world, w) for w in self.ws]
         self.counts_of = pointer_array([v["counts"] for v in self.views], self.device)
         self.x_recv_of = pointer_array(self.x_recv, self.device)
@@ -601,7 +614,7 @@ def workspace_views(dm: MoeDims, ws: torch.Tensor) -> dict:
         "token_of_row": view(L["token_of_row"], cap, torch.int32, (cap,)),
         "x_perm": view(L["x_perm"], cap * d, torch.bfloat16, (cap, d)),
         "h_perm": view(L["h_perm"], cap * I, torch.bfloat16, (cap, I)),
-        "y_perm": view(L["y_perm"], cap * d, torch.bfloat16, (cap, d)),
+        "y_perm": view(L["y_perm"], cap * d, torch.float32, (cap, d)),
         "h_shared": view(L["h_shared"], T * S * I, torch.bfloat16, (T, S * I)),
         "y_shared": view(L["y_shared"], T * d, torch.float32, (T, d)),
     }
@@ -621,10 +634,10 @@ def train_workspace_views(dm: MoeDims, ws: torch.Tensor) -> dict:
 
     bf, f32 = torch.bfloat16, torch.float32
     v.update({
-        "g_perm": view(L["g_perm"], cap * I, bf, (cap, I)),
-        "u_perm": view(L["u_perm"], cap * I, bf, (cap, I)),
-        "g_shared": view(L["g_shared"], T * S * I, bf, (T, S * I)),
-        "u_shared": view(L["u_shared"], T * S * I, bf, (T, S * I)),
+        "g_perm": view(L["g_perm"], cap * I, f32, (cap, I)),
+        "u_perm": view(L["u_perm"], cap * I, f32, (cap, I)),
+        "g_shared": view(L["g_shared"], T * S * I, f32, (T, S * I)),
+        "u_shared": view(L["u_shared"], T * S * I, f32, (T, S * I)),
         "dy_perm": view(L["dy_perm"], cap * d, bf, (cap, d)),
         "dw": view(L["dw"], T * k, f32, (T, k)),
         "dz": view(L["dz"], T * E, f32, (T, E)),
@@ -708,9 +721,11 @@ class MoELayer:
                       self.ws1, self.ws3, self.ws2, y, self.train_workspace(T), stream)
         return y
 
-    def alloc_grads(self, T: int) -> dict:
+    def alloc_grads(self, T: int, dtype=torch.bfloat16) -> dict:
+        """Gradient buffers: dx and the expert weight gradients in ``dtype``
+        (bf16 or fp32), the gate's gradient in fp32."""
         c, dev = self.cfg, self.device
-        bf = dict(dtype=torch.bfloat16, device=dev)
+        bf = dict(dtype=dtype, device=dev)
         return {"dx": torch.empty((T, c.d), **bf),
                 "dw_gate": torch.empty((c.E, c.d), dtype=torch.float32, device=dev),
                 "dw1": torch.empty((c.E, c.I, c.d), **bf), "dw3": torch.empty((c.E, c.I, c.d), **bf),

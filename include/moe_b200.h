@@ -165,28 +165,30 @@ int moe_permute(const moe_dims* dims, const int32_t* topk_idx,
  *   offsets [E+1]      int32 segment starts (moe_permute output)
  *   w1, w3  [E, I, d]  bf16;  w2 [E, d, I] bf16
  *   h_perm  [cap, I]   bf16 out: silu(x w1^T) * (x w3^T) for every segment row
- *   y_perm  [cap, d]   bf16 out: h w2^T for every segment row
+ *   y_perm  [cap, d]   fp32 out: h w2^T for every segment row (the fp32
+ *                      accumulators, not rounded: a bf16 copy would round a
+ *                      dominant expert's output twice on its way into y)
  * Rows outside [0, offsets[E]) are neither read nor written.  Padding rows are
  * computed like the others (zero rows give zero outputs).  No workspace.
  * ---------------------------------------------------------------------- */
 int moe_grouped_swiglu(const moe_dims* dims, const moe_bf16* x_perm,
                        const int32_t* offsets, const moe_bf16* w1,
                        const moe_bf16* w3, const moe_bf16* w2,
-                       moe_bf16* h_perm, moe_bf16* y_perm, void* stream);
+                       moe_bf16* h_perm, float* y_perm, void* stream);
 
 /* ------------------------------------------------------------------------
  * moe_combine -- weighted un-permute and shared-expert add.
  * Technical Report, Method: output = shared experts (weight 1) + the k routed
  * experts weighted by the gate.
  *
- *   y_perm   [cap, d]  bf16 routed expert outputs per segment row
+ *   y_perm   [cap, d]  fp32 routed expert outputs per segment row
  *   row_of   [T*k]     int32 row of each (token, slot) pair
  *   topk_w   [T, k]    fp32 weights
  *   y_shared [T, d]    fp32 sum of the shared experts' outputs (may be NULL)
  *   y        [T, d]    bf16 out: y[t] = y_shared[t] + sum_j w[t,j] y_perm[row_of[t*k+j]]
  * The sum runs in fp32, slot j in ascending order, and is rounded once.
  * ---------------------------------------------------------------------- */
-int moe_combine(const moe_dims* dims, const moe_bf16* y_perm,
+int moe_combine(const moe_dims* dims, const float* y_perm,
                 const int32_t* row_of, const float* topk_w,
                 const float* y_shared, moe_bf16* y, void* stream);
 
@@ -215,7 +217,7 @@ typedef struct moe_ws_layout {
   size_t permute_scratch; /* moe_permute_workspace_size() bytes            */
   size_t x_perm;          /* bf16 [cap, d]                                 */
   size_t h_perm;          /* bf16 [cap, I]                                 */
-  size_t y_perm;          /* bf16 [cap, d]                                 */
+  size_t y_perm;          /* fp32 [cap, d]                                 */
   size_t h_shared;        /* bf16 [T, S*I]; column s*I + i = shared expert s */
   size_t y_shared;        /* fp32 [T, d]   sum of the shared experts        */
   size_t total;           /* = moe_workspace_size()                        */
@@ -235,7 +237,10 @@ int moe_forward(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
  * in the backward pass.
  *
  * moe_forward_train is moe_forward that also keeps the gate/up
- * pre-activations (g = w1 x, u = w3 x, bf16) for the backward.  Its workspace
+ * pre-activations (g = w1 x, u = w3 x) for the backward, in fp32: they feed
+ * only the SwiGLU backward's arithmetic, not a tensor-core operand, and bf16
+ * copies of them would cost the shared experts' weight gradients about 1 %
+ * of their rms in accuracy.  Its workspace
  * (moe_train_workspace_size() bytes, 256-byte aligned) starts with the
  * forward layout (same offsets as moe_forward_layout) and adds the regions
  * of moe_train_layout.
@@ -245,6 +250,11 @@ int moe_forward(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
  *   dx [T, d] bf16, dw_gate [E, d] fp32, dw1, dw3 [E, I, d], dw2 [E, d, I],
  *   dws1, dws3 [S, I, d], dws2 [S, d, I] (bf16; every element is written,
  *   experts that received no token get zero).
+ * moe_backward_f32 is the same computation with dx and every expert weight
+ * gradient written in fp32: the tensor-core accumulators and the fp32 sum of
+ * dx are stored unrounded (moe_backward's outputs are exactly their bf16
+ * roundings, to nearest even).  Use it where the gradients are accumulated or
+ * applied in fp32; it writes twice the bytes.
  * The routing choice of the forward is held fixed; the bias only enters the
  * selection key and gets no gradient.  Gradients flow through the combine
  * weights, the renormalisation and the softmax into w_gate and x.  Extra
@@ -252,10 +262,10 @@ int moe_forward(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
  * ---------------------------------------------------------------------- */
 typedef struct moe_train_layout {
   moe_ws_layout fwd;    /* the forward intermediates (moe_forward_layout)  */
-  size_t g_perm;        /* bf16 [cap, I]  gate pre-activations             */
-  size_t u_perm;        /* bf16 [cap, I]  up pre-activations               */
-  size_t g_shared;      /* bf16 [T, S*I]                                   */
-  size_t u_shared;      /* bf16 [T, S*I]                                   */
+  size_t g_perm;        /* fp32 [cap, I]  gate pre-activations             */
+  size_t u_perm;        /* fp32 [cap, I]  up pre-activations               */
+  size_t g_shared;      /* fp32 [T, S*I]                                   */
+  size_t u_shared;      /* fp32 [T, S*I]                                   */
   size_t dy_perm;       /* bf16 [cap, d]  w * dy per segment row            */
   size_t dw;            /* fp32 [T, k]    gradient of the combine weights   */
   size_t dz;            /* fp32 [T, E]    gradient of the gate logits       */
@@ -282,6 +292,12 @@ int moe_backward(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
                  moe_bf16* dx, float* dw_gate, moe_bf16* dw1, moe_bf16* dw3,
                  moe_bf16* dw2, moe_bf16* dws1, moe_bf16* dws3, moe_bf16* dws2,
                  void* stream);
+int moe_backward_f32(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
+                     const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
+                     const moe_bf16* ws1, const moe_bf16* ws3, const moe_bf16* ws2,
+                     const moe_bf16* dy, void* workspace, size_t workspace_bytes, float* dx,
+                     float* dw_gate, float* dw1, float* dw3, float* dw2, float* dws1,
+                     float* dws3, float* dws2, void* stream);
 
 /* ------------------------------------------------------------------------
  * moe_dense_swiglu -- the dense SwiGLU FFN of the model's first layer
@@ -442,19 +458,19 @@ int moe_ep_dispatch(const moe_dims* dims, int world, int rank, const moe_bf16* x
  *   x_recv   [recv_cap, d] this rank's receive buffer
  *   w1, w3   [El, I, d], w2 [El, d, I] bf16: this rank's experts only
  *   ws1, ws3 [S, I, d], ws2 [S, d, I] shared experts (NULL iff S == 0)
- *   y_recv   [recv_cap, d] bf16 out: expert outputs per receive row
+ *   y_recv   [recv_cap, d] fp32 out: expert outputs per receive row
  * Rows at or after the last segment are neither read nor written. */
 int moe_ep_experts(const moe_dims* dims, int world, const moe_bf16* x,
                    const moe_bf16* x_recv, const moe_bf16* w1, const moe_bf16* w3,
                    const moe_bf16* w2, const moe_bf16* ws1, const moe_bf16* ws3,
-                   const moe_bf16* ws2, moe_bf16* y_recv, void* workspace,
+                   const moe_bf16* ws2, float* y_recv, void* workspace,
                    size_t workspace_bytes, void* stream);
 
 /* moe_ep_combine --
- *   y_recv  device array [W] of the ranks' expert-output buffers
+ *   y_recv  device array [W] of the ranks' fp32 expert-output buffers
  *   y       [T, d] bf16 out
  * Same arithmetic as moe_combine; a pair that was not sent contributes 0. */
-int moe_ep_combine(const moe_dims* dims, int world, const moe_bf16* const* y_recv,
+int moe_ep_combine(const moe_dims* dims, int world, const float* const* y_recv,
                    moe_bf16* y, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------

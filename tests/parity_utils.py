@@ -8,8 +8,10 @@ workload specification fixes):
   * fp32 router probabilities and weights: relative error <= 1e-5;
   * integer / index outputs of the permutation: bit-exact, against the oracle
     run on the GPU's own routing;
-  * bf16 intermediates (h, y_perm): every element within 2^-8 of its own
-    magnitude (one bf16 rounding plus fp32 accumulation) plus 1e-3 rms;
+  * bf16 intermediates (h): every element within 2^-8 of its own magnitude
+    (one bf16 rounding plus fp32 accumulation) plus 1e-3 rms; fp32 sums of
+    exact bf16 products (y_perm and y_shared against the oracle fed the GPU's
+    own bf16 h): within 1e-5 of the sum of the products' magnitudes;
   * the layer output y (bf16): max |gpu - oracle| <= 2e-2 * rms(oracle) on the
     workload configurations.  Shapes outside them (edge cases with heavier
     output tails or cancelling terms, e.g. k = 8 with one shared expert, or no
@@ -17,18 +19,24 @@ workload specification fixes):
     own bf16 rounding (2^-8 |y|) plus the bf16 rounding of every routed
     output it sums (2^-8 sum_j w_j |o_j|), plus 1e-2 rms(y) for the rounding
     of h carried through the down projection.
-  * gradients of the backward (bf16 dx, dW; fp32 dWg): the 2e-2 * rms bound
-    is below what any bf16 answer can reach for them -- the routed experts'
-    weight gradients are sums over ~12 tokens dominated by single large
-    products (max |dW| ~ 17 rms), and even the exactly-rounded bf16 value of
-    the fp64 gradient is off by ~6 % of rms there.  Every element must lie
-    within three bf16 roundings of its own magnitude (output, and the two
-    rounded inputs of its dominant product) plus 2e-2 rms.  For the routed
-    experts' weight gradients (sums whose products can nearly cancel) the
-    bound also carries kappa * u * A, with A = sum |a_t||b_t| over the
-    element's products, kappa the number of bf16 roundings feeding a product
-    and u = 2^-8 the bf16 unit roundoff; a CPU emulation of the bf16 storage
-    points reproduces the GPU's values at the worst elements.
+    Where even the correctly rounded bf16 value of the exact output is more
+    than 2e-2 rms away at some element (a large output where the bf16
+    spacing is coarse: 0.0625 above 8), no bf16 answer can meet the bound;
+    then every element must lie within 2e-2 rms plus its own unavoidable
+    rounding |bf16(ref) - ref|.
+  * gradients of the backward on the workload configurations: the fp32
+    outputs (moe_backward_f32) of dx, dWg and the shared experts' weight
+    gradients within 2e-2 rms; the bf16 outputs (moe_backward) are exactly
+    their roundings to nearest even.  The routed experts' weight gradients
+    are sums over ~12 tokens dominated by single large products; with bf16
+    MMA operands (w*dy, h, dG, dU: each one rounding) even exact arithmetic
+    misses 2e-2 rms there (a CPU emulation on the same inputs shows it, and
+    the check falls back to the spec bound wherever the emulation meets
+    it).  Their bound is the arithmetic's: every element within two bf16
+    roundings of its own magnitude plus 2e-2 rms plus kappa * u * A, with
+    A = sum |a_t||b_t| over the element's products, kappa the number of bf16
+    roundings feeding a product and u = 2^-8 the bf16 unit roundoff.
+    Off-spec shapes hold every gradient to that arithmetic bound.
 """
 import numpy as np
 import torch
@@ -84,14 +92,48 @@ def check_bf16_elementwise(got, ref, what):
     return float(err.max()) if err.size else 0.0
 
 
+def check_fp32_sum(got, ref, abs_sum, what):
+    """An fp32 tensor-core sum of exact bf16 products: every element within
+    1e-5 of the sum of its products' magnitudes (fp32 accumulation over a few
+    thousand terms is ~100 times tighter than this)."""
+    got, ref = to_np(got), np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    err = np.abs(got - ref)
+    bound = 1e-5 * np.asarray(abs_sum) + 1e-30
+    worst = np.unravel_index(np.argmax(err / bound), err.shape) if err.size else None
+    assert np.all(err <= bound), f"{what}: worst at {worst}: got {got[worst]} ref {ref[worst]}"
+    return float(err.max()) if err.size else 0.0
+
+
+def bf16_round(a):
+    """The nearest bf16 value of every element (round to nearest even)."""
+    return torch.tensor(np.asarray(a, dtype=np.float64)).float().to(torch.bfloat16).double().numpy()
+
+
 def check_output(y_gpu, y_ref, what="y", spec=True, routed_abs=None):
+    """Layer output against the oracle.  spec: max |gpu - oracle| <= 2e-2 rms.
+    Where that fails, it must be because no bf16 answer can meet it: the
+    correctly rounded exact value itself is more than 2e-2 rms away at some
+    element (a large output where the bf16 spacing is coarse).  Then every
+    element must lie within 2e-2 rms plus its own unavoidable rounding
+    |bf16(ref) - ref|."""
     y_gpu, y_ref = to_np(y_gpu), np.asarray(y_ref, dtype=np.float64)
     assert np.isfinite(y_gpu).all(), f"{what}: non-finite values"
     r = rms(y_ref)
     diff = np.abs(y_gpu - y_ref)
     err = float(diff.max()) if y_ref.size else 0.0
     if spec:
-        assert err <= Y_RMS_FRAC * r + 1e-30, f"{what}: max err {err:.4e} > {Y_RMS_FRAC} * rms {r:.4e}"
+        if err > Y_RMS_FRAC * r:
+            floor = np.abs(bf16_round(y_ref) - y_ref)
+            assert floor.max() > Y_RMS_FRAC * r, (
+                f"{what}: max err {err:.4e} > {Y_RMS_FRAC} * rms {r:.4e} "
+                f"(the correctly rounded answer is within it: {floor.max() / r:.4f} rms)")
+            worst = np.unravel_index(np.argmax(diff - floor), diff.shape)
+            assert np.all(diff <= Y_RMS_FRAC * r + floor), (
+                f"{what}: worst at {worst}: got {y_gpu[worst]} ref {y_ref[worst]} "
+                f"beyond 2e-2 rms plus its own rounding {floor[worst]:.4e}")
+            print(f"{what}: max err {err / r:.4f} rms; the correctly rounded exact answer "
+                  f"is already {floor.max() / r:.4f} rms off at its worst element")
     else:
         extra = 0.0 if routed_abs is None else BF16_REL * np.asarray(routed_abs)
         bound = BF16_REL * np.abs(y_ref) + extra + 1e-2 * r + 1e-30
@@ -105,16 +147,36 @@ def bf16_floor(ref):
     r = rms(ref)
     if r == 0:
         return 0.0
-    rounded = torch.tensor(ref, dtype=torch.float32).to(torch.bfloat16).double().numpy()
-    return float(np.abs(rounded - ref).max() / r)
+    return float(np.abs(bf16_round(ref) - ref).max() / r)
 
 
-def check_grad(got, ref, what, abs_sum=None, kappa=0):
+def rel_err(got, ref, scale=None):
+    """max |got - ref| / rms(ref) (or / scale)."""
+    got, ref = to_np(got), np.asarray(ref, dtype=np.float64)
+    r = rms(ref) if scale is None else scale
+    return float(np.abs(got - ref).max()) / r if r > 0 and ref.size else 0.0
+
+
+def check_spec(got, ref, what):
+    """The workload specification's bound: max |gpu - oracle| <= 2e-2 rms."""
+    got, ref = to_np(got), np.asarray(ref, dtype=np.float64)
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    r = rms(ref)
+    err = float(np.abs(got - ref).max()) if ref.size else 0.0
+    assert err <= Y_RMS_FRAC * r + 1e-30, f"{what}: max err {err / r:.4f} rms > {Y_RMS_FRAC}"
+    return err / r if r > 0 else 0.0
+
+
+def check_grad(got, ref, what, abs_sum=None, kappa=0, rounded_output=True):
+    """The arithmetic's bound for a gradient: the roundings of its own output
+    (when bf16) and of the two inputs of its dominant product, 2^-8 of its
+    magnitude each, plus 2e-2 rms, plus kappa * 2^-8 * abs_sum for sums of
+    products that can nearly cancel."""
     got, ref = to_np(got), np.asarray(ref, dtype=np.float64)
     assert np.isfinite(got).all(), f"{what}: non-finite values"
     r = rms(ref)
     diff = np.abs(got - ref)
-    bound = 3 * BF16_REL * np.abs(ref) + Y_RMS_FRAC * r + 1e-30
+    bound = (3 if rounded_output else 2) * BF16_REL * np.abs(ref) + Y_RMS_FRAC * r + 1e-30
     if abs_sum is not None:
         bound = bound + kappa * BF16_REL * np.asarray(abs_sum)
     worst = np.unravel_index(np.argmax(diff / bound), diff.shape) if diff.size else None

@@ -170,7 +170,7 @@ GEMM_CASES = [
 def _grouped(dm, x_perm, offsets, g):
     cap = M.capacity(dm)
     h = torch.full((cap, dm.I), float("nan"), dtype=torch.bfloat16, device=DEV)
-    y = torch.full((cap, dm.d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    y = torch.full((cap, dm.d), float("nan"), dtype=torch.float32, device=DEV)
     M.grouped_swiglu(dm, x_perm, offsets, g["w1"], g["w3"], g["w2"], h, y)
     return h, y
 
@@ -196,9 +196,9 @@ def test_grouped_swiglu_parity(name, cfg, T, align):
         xe = xp[a:b].cpu()
         o_ref, h_ref, _, _ = O.swiglu_expert(xe, inp["w1"][e], inp["w3"][e], inp["w2"][e])
         PU.check_bf16_elementwise(h[a:b], h_ref, f"h_perm expert {e}")
-        # the down GEMM against the oracle fed with the GPU's own bf16 h
-        o_from_h = PU.to_np(h[a:b]) @ inp["w2"][e].double().numpy().T
-        PU.check_bf16_elementwise(y[a:b], o_from_h, f"y_perm expert {e}")
+        # the down GEMM (fp32 out) against the oracle fed with the GPU's own bf16 h
+        hg, w2 = PU.to_np(h[a:b]), inp["w2"][e].double().numpy()
+        PU.check_fp32_sum(y[a:b], hg @ w2.T, np.abs(hg) @ np.abs(w2).T, f"y_perm expert {e}")
 
 
 # ------------------------------------------------------------------ combine
@@ -208,7 +208,7 @@ def test_combine_parity():
     dm = M.dims(T, d, E, k, 64, 2, 16)
     cap = M.capacity(dm)
     gen = torch.Generator().manual_seed(3)
-    y_perm = torch.randn((cap, d), generator=gen).to(torch.bfloat16)
+    y_perm = torch.randn((cap, d), generator=gen)
     rows = torch.randperm(cap, generator=gen)[:T * k].to(torch.int32)
     w = torch.rand((T, k), generator=gen)
     w = w / w.sum(1, keepdim=True)
@@ -291,11 +291,13 @@ def test_forward_deterministic():
 # ------------------------------------------------------------------ full-size configurations
 
 @pytest.mark.parametrize("cfg,n_sample,seed",
-                         [(DECODE, 24, 1), (PREFILL_BALANCED, 12, 2), (PREFILL_SKEWED, 12, 3)],
+                         [(DECODE, 128, 1), (PREFILL_BALANCED, 1024, 2),
+                          (PREFILL_SKEWED, 1024, 3)],
                          ids=["decode", "prefill_balanced", "prefill_skewed"])
 def test_forward_full_size_sampled(cfg, n_sample, seed):
     """The full configuration on the device: the whole routing and permutation
-    are compared; the output on a seeded sample of tokens (per-token oracle)."""
+    are compared; the output on a seeded sample of tokens (per-token oracle;
+    every token of the decode batch, 1024 of a prefill batch)."""
     inp = make_inputs(cfg, device=DEV)
     layer = M.MoELayer(inp)
     y = layer(inp["x"])
@@ -315,3 +317,51 @@ def test_forward_full_size_sampled(cfg, n_sample, seed):
     toks = np.sort(rng.choice(cfg.T, size=n_sample, replace=False))
     ref = O.forward_tokens(host, toks, idx=idx_gpu[toks])
     PU.check_output(y[torch.as_tensor(toks, device=DEV)], ref["y"], "y (sampled)")
+
+
+@pytest.mark.parametrize("cfg", [DECODE, PREFILL_BALANCED, PREFILL_SKEWED],
+                         ids=["decode", "prefill_balanced", "prefill_skewed"])
+def test_forward_full_size_every_segment(cfg):
+    """Every tile of both grouped GEMMs at the full configuration (one-CTA
+    kernels at decode, CTA pairs at prefill): h_perm and y_perm of every
+    non-empty expert segment, and the shared experts' h and fp32 y, each
+    against the oracle's SwiGLU expert fed the GPU's own permuted rows (for
+    the down projection, the GPU's own bf16 h: exactly what that GEMM read).
+    Segment rows beyond a segment's tokens (padding) must be exactly zero."""
+    inp = make_inputs(cfg, device=DEV)
+    layer = M.MoELayer(inp)
+    layer(inp["x"])
+    torch.cuda.synchronize()
+    assert M.device_status() == M.MOE_OK
+    v = M.workspace_views(layer.dims(cfg.T), layer.workspace(cfg.T))
+    off = v["offsets"].cpu().numpy()
+    counts = v["counts"].cpu().numpy()
+    done = 0
+    for e in range(cfg.E):
+        a, b = int(off[e]), int(off[e + 1])
+        if a == b:
+            continue
+        xe = v["x_perm"][a:b]
+        _, h_ref, _, _ = O.swiglu_expert(xe, inp["w1"][e], inp["w3"][e], inp["w2"][e])
+        PU.check_bf16_elementwise(v["h_perm"][a:b], h_ref, f"h_perm expert {e}")
+        w2 = inp["w2"][e].double().cpu().numpy()
+        hg = PU.to_np(v["h_perm"][a:b])
+        PU.check_fp32_sum(v["y_perm"][a:b], hg @ w2.T, np.abs(hg) @ np.abs(w2).T,
+                          f"y_perm expert {e}")
+        pad = slice(a + int(counts[e]), b)
+        assert not v["h_perm"][pad].any() and not v["y_perm"][pad].any(), f"padding of {e}"
+        done += 1
+    assert done == int((counts > 0).sum())
+    S, I = cfg.S, cfg.I
+    h_sh = v["h_shared"]
+    y_ref = np.zeros((cfg.T, cfg.d))
+    y_abs = np.zeros((cfg.T, cfg.d))
+    for s_ in range(S):
+        _, h_ref, _, _ = O.swiglu_expert(inp["x"], inp["ws1"][s_], inp["ws3"][s_], inp["ws2"][s_])
+        hs = h_sh[:, s_ * I:(s_ + 1) * I]
+        PU.check_bf16_elementwise(hs, h_ref, f"h_shared expert {s_}")
+        w2 = inp["ws2"][s_].double().cpu().numpy()
+        hg = PU.to_np(hs)
+        y_ref += hg @ w2.T
+        y_abs += np.abs(hg) @ np.abs(w2).T
+    PU.check_fp32_sum(v["y_shared"], y_ref, y_abs, "y_shared")

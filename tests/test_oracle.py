@@ -588,3 +588,23 @@ def test_ep_exchange_reproduces_the_layer_output(W, align):
             y[t] += routes[s]["w"][t, j] * outs[L["owner"][s][p]][L["row"][s][p]]
         want = O.forward(dict(host, x=x, T=x.shape[0]), align=align)["y"]
         np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-12)
+
+
+def test_bf16_emulation_without_rounding_is_the_oracle_backward():
+    """The backward tests' emulation of the bf16 MMA operands, with the
+    rounding switched off, must give the oracle's routed weight gradients
+    (it restates them from the forward's intermediates, not through
+    swiglu_expert_backward); with bf16 rounding it must differ."""
+    import bf16_emulation as EM
+    cfg = small_config(T=40, d=64, E=8, k=2, I=64)
+    inp = make_inputs(cfg)
+    inp["dy"] = torch.randn((40, 64), generator=torch.Generator().manual_seed(2)).to(torch.bfloat16)
+    f = O.forward(inp)
+    b = O.backward(inp, inp["dy"], f)
+    ex = list(range(cfg.E))
+    exact = EM.routed_weight_grads(inp, f, b, ex, rnd=lambda a: np.asarray(a, dtype=np.float64))
+    rounded = EM.routed_weight_grads(inp, f, b, ex)
+    for name in ("dw1", "dw3", "dw2"):
+        for e in ex:
+            np.testing.assert_allclose(exact[name][e], b[name][e], rtol=0, atol=1e-12)
+        assert max(np.abs(rounded[name][e] - b[name][e]).max() for e in ex) > 0
