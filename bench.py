@@ -902,6 +902,8 @@ def run_ep(args):
                 "d2h_bytes_per_step": W * T * d * 2},
         "gpu_launches": W * ep_kernels(T) * args.steps,
     }
+    if args.micro > 1:
+        line["overlap"] = ep_overlap_measurement(args, inp, xs, W, T, dev, stream, phase_ms)
     if not args.no_cpu_baseline:
         n, secs = oracle_sample(inp, args.cpu_tokens)
         line["cpu_baseline"] = {"value": n / secs, "unit": "tokens/s", "cores": cpu_threads(),
@@ -909,6 +911,155 @@ def run_ep(args):
                                 "sample": f"{n} seeded tokens of rank 0's batch, fp64 numpy "
                                           f"oracle (forward; the exchange does not change it), "
                                           f"{secs:.1f} s"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def ep_overlap_measurement(args, inp, xs, W, T, dev, stream, phase_ms):
+    """The expert-parallel step with every rank's batch split into
+    --micro microbatches, each chain (route, dispatch, experts, combine) on
+    its own stream: timed against the same calls issued microbatch after
+    microbatch, with a per-microbatch phase timeline of one untimed step."""
+    from fine_grained_moe_fp32_b200 import moe as M
+    from fine_grained_moe_fp32_b200.overlap import EPOverlap
+    ov = EPOverlap(inp, W, T, args.micro, args.align, dev)
+    ys = [torch.empty((T, inp["cfg"].d), dtype=torch.bfloat16, device=dev) for _ in range(W)]
+    for _ in range(args.warmup):
+        ov(xs, ys)
+        ov.serial(xs, ys)
+    torch.cuda.synchronize(dev)
+
+    def timed(fn):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn(xs, ys)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / args.steps
+
+    ovl_ms = timed(ov)
+    ser_ms = timed(ov.serial)
+    # timeline of one overlapped step: every microbatch's phase boundaries
+    t0 = torch.cuda.Event(enable_timing=True)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in ov.sizes]
+    t0.record(stream)
+    ov(xs, ys, events=evs)
+    torch.cuda.synchronize(dev)
+    if M.device_status() != M.MOE_OK:
+        raise SystemExit("device status after the overlapped steps")
+    names = ("route", "dispatch", "experts", "combine")
+    timeline = [{n: [round(t0.elapsed_time(e[i]), 4), round(t0.elapsed_time(e[i + 1]), 4)]
+                 for i, n in enumerate(names)} for e in evs]
+    # phase sum of the microbatched work: each microbatch's own phases, timed
+    # one after the other (untimed pass, events between phases)
+    sum_micro = 0.0
+    for i, ep in enumerate(ov.parts):
+        xi = ov._slices(xs, i)
+        yi = ov._slices(ys, i)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        e[0].record(stream)
+        ep.route(xi)
+        e[1].record(stream)
+        ep.dispatch(xi)
+        e[2].record(stream)
+        ep.experts_step(xi)
+        e[3].record(stream)
+        ep.combine(yi)
+        e[4].record(stream)
+        torch.cuda.synchronize(dev)
+        sum_micro += e[0].elapsed_time(e[4])
+    return {"microbatches": ov.sizes, "overlapped_ms_per_step": ovl_ms,
+            "serial_ms_per_step": ser_ms, "sum_of_microbatch_phases_ms": sum_micro,
+            "sum_of_unsplit_phases_ms": sum(phase_ms.values()),
+            "hidden_fraction_vs_serial": 1.0 - ovl_ms / ser_ms,
+            "timeline_ms": timeline,
+            "note": "each microbatch's route -> dispatch -> experts -> combine on its own "
+                    "stream; serial = the same calls one microbatch after the other"}
+
+
+def run_paired(args):
+    """One pipeline stage executing the overlapped interleaved-1F1B step
+    list (one warm-up forward, then a forward of microbatch m+1 and the
+    backward of microbatch m together on two streams, then the last
+    backward) at the workload's microbatch size, timed against the same
+    passes run one at a time."""
+    from fine_grained_moe_fp32_b200 import moe as M
+    from fine_grained_moe_fp32_b200.overlap import PipelineStage
+    from fine_grained_moe_fp32_b200.pipeline_schedule import interleaved_1f1b
+    world, rank, local = dist_setup()
+    if world > 1:
+        raise SystemExit("--paired runs one pipeline stage on one GPU; run it without torchrun")
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cfg = workload(args)
+    if not cfg.grad:
+        cfg = dataclasses.replace(CONFIGS[4], T=cfg.T, name=CONFIGS[4].name)
+    T, Mn = cfg.T, max(2, args.micro)
+    inp = make_inputs(cfg, device=dev)
+    layer = M.MoELayer(inp, align=args.align, device=dev)
+    xs = [inp["x"]] + [make_inputs(cfg, device=dev, seed=1000 + m, weights=False)["x"]
+                       for m in range(1, Mn)]
+    dys = [inp["dy"]] + [make_inputs(cfg, device=dev, seed=2000 + m, weights=False)["dy"]
+                         for m in range(1, Mn)]
+    steps = interleaved_1f1b(1, 1, Mn, overlap=True)[0]
+    stage = PipelineStage([layer], T, grad_dtype=torch.bfloat16)
+    # one gradient buffer set: the backwards run one after the other on their stream
+    g = layer.alloc_grads(T)
+    grads = {(m, 0): g for m in range(Mn)}
+    ys = {(m, 0): torch.empty((T, cfg.d), dtype=torch.bfloat16, device=dev) for m in range(Mn)}
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        stage.run(steps, xs, dys, grads, ys)
+        stage.sequential(steps, xs, dys, grads, ys)
+    torch.cuda.synchronize(dev)
+
+    def timed(fn):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn(steps, xs, dys, grads, ys)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / args.steps
+
+    sampler = ClockSampler(local)
+    time.sleep(0.15)
+    t0 = time.time()
+    ovl = timed(stage.run)
+    t1 = time.time()
+    clocks = sampler.stop(t0, t1)
+    seq = timed(stage.sequential)
+    if M.device_status() != M.MOE_OK:
+        raise SystemExit("device status after the paired steps")
+    flops = sum(train_gemm_flops(cfg, T).values()) * Mn
+    peaks, peak_src = load_peaks()
+    ach = flops / (ovl / 1e3) / 1e12
+    line = {
+        "metric": "MoE-layer fwd+bwd tokens/s through one pipeline stage running the overlapped "
+                  "interleaved-1F1B steps (bf16, d=5120, 128E top-6 + 2 shared)",
+        "value": Mn * T / (ovl / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ovl, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) tokens and upstream gradients, N(0,0.02) weights)",
+        "config": {"workload": f"paired_1f1b_{cfg.name}_x{Mn}", "T_per_microbatch": T,
+                   "microbatches": Mn, "d": cfg.d, "E": cfg.E, "k": cfg.k, "S": cfg.S,
+                   "I": cfg.I, "schedule": [[f"{k}{m}" for k, m, _ in st] for st in steps],
+                   "parallelism": "one pipeline stage (P=1, V=1) on one GPU"},
+        "roofline": {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+                     "kernel": "whole stage (all GEMM phases of every pass)",
+                     "peak_source": f"{peak_src} (bf16_tflops)", "traffic": None,
+                     "algorithmic_per_launch": flops},
+        "sequential_ms_per_step": seq, "overlapped_ms_per_step": ovl,
+        "hidden_fraction": 1.0 - ovl / seq, "clocks": clocks,
+        "e2e": None,
+        "gpu_launches": Mn * (forward_kernels(T) + BWD_KERNELS) * args.steps,
+    }
     print(json.dumps(line), flush=True)
     return 0
 
@@ -934,6 +1085,12 @@ def main(argv=None):
                     help="expert parallelism over this many ranks emulated on one GPU")
     ap.add_argument("--dense", action="store_true",
                     help="time the first layer's dense SwiGLU FFN instead of the MoE layer")
+    ap.add_argument("--micro", type=int, default=0,
+                    help="--ep: also time the step with every rank's batch split into this many "
+                         "microbatches on their own streams; --paired: microbatches (default 4)")
+    ap.add_argument("--paired", action="store_true",
+                    help="one pipeline stage running the overlapped interleaved-1F1B steps "
+                         "(training workload, forward and backward of two microbatches together)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -943,6 +1100,12 @@ def main(argv=None):
         return run_dense(args)
     if args.ep:
         return run_ep(args)
+    if args.paired:
+        if args.micro == 0:
+            args.micro = 4
+        if args.config == 1:
+            args.config = 4
+        return run_paired(args)
     return run_ours(args)
 
 

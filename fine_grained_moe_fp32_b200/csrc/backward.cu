@@ -12,6 +12,7 @@
 #include <cuda_bf16.h>
 
 #include "moe_internal.h"
+#include "checks.cuh"
 
 namespace moe {
 namespace {
@@ -46,7 +47,7 @@ combine_bwd_kernel(const uint16_t* __restrict__ dy, const float* __restrict__ y_
     const int r = row_of[(size_t)t * k + j];
     const float w = topk_w[(size_t)t * k + j];
     float part = 0.f;
-    if (r >= 0 && r < cap) {
+    if (MOE_CHECK(r >= -1 && r < cap) && r >= 0 && r < cap) {
       const float4* yr = reinterpret_cast<const float4*>(y_perm + (size_t)r * d);
       uint4* out = reinterpret_cast<uint4*>(dy_perm + (size_t)r * d);
 #pragma unroll
@@ -321,7 +322,7 @@ unpermute_bwd_kernel(const float* __restrict__ dx_shared, const float* __restric
   __shared__ int rows[8];
   if (threadIdx.x < k) {
     const int r = row_of[(size_t)t * k + threadIdx.x];
-    rows[threadIdx.x] = (r >= 0 && r < cap) ? r : -1;
+    rows[threadIdx.x] = (MOE_CHECK(r >= -1 && r < cap) && r >= 0 && r < cap) ? r : -1;
   }
   __syncthreads();
   for (int v = threadIdx.x; v < d / 8; v += kCbThreads) {
@@ -417,3 +418,5 @@ cudaError_t launch_backward_misc_post(const Shape& s, const BackwardMiscArgs& a,
 }
 
 }  // namespace moe
+
+MOE_CHECKS_UNIT(backward)

@@ -171,7 +171,7 @@ BalancePlan plan(const Shape& s, int seq_len) {
 }  // namespace
 
 size_t balance_workspace_bytes(const Shape& s, int seq_len) {
-  return plan(s, seq_len).total;
+  return plan(s, seq_len).total + kGuardBytes;
 }
 
 cudaError_t launch_balance_stats(const Shape& s, int seq_len, const float* probs,

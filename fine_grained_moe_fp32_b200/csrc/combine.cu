@@ -14,6 +14,7 @@
 #include <cuda_bf16.h>
 
 #include "moe_internal.h"
+#include "checks.cuh"
 
 namespace moe {
 namespace {
@@ -39,6 +40,7 @@ struct LocalRows {
   int64_t cap;
   __device__ const float* row(size_t p, int d) const {
     const int r = row_of[p];
+    if (!MOE_CHECK(r >= -1 && r < cap)) return nullptr;  // -1: a pair that was skipped
     return (r >= 0 && r < cap) ? y_perm + (size_t)r * d : nullptr;
   }
 };
@@ -53,6 +55,7 @@ struct OwnerRows {
   int64_t cap;
   __device__ const float* row(size_t p, int d) const {
     const int e = topk_idx[p], r = remote_row[p];
+    if (!MOE_CHECK(r >= -1 && r < cap)) return nullptr;  // -1: a pair that was not sent
     if (e < 0 || e >= E || r < 0 || r >= cap) return nullptr;
     const float* b = y_recv[e / El];
     return (reinterpret_cast<uintptr_t>(b) & 15) ? nullptr : b + (size_t)r * d;
@@ -130,3 +133,5 @@ cudaError_t launch_ep_combine(const Shape& s, int world, const float* const* y_r
 }
 
 }  // namespace moe
+
+MOE_CHECKS_UNIT(combine)

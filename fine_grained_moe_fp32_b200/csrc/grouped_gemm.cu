@@ -30,6 +30,7 @@
 #include <cudaTypedefs.h>
 
 #include "moe_internal.h"
+#include "checks.cuh"
 #include "ptx_sm100.cuh"
 
 namespace moe {
@@ -71,6 +72,7 @@ struct GemmParams {
   float* u_shared;
   unsigned int* status;
   uint64_t wait_limit_ns;
+  int64_t rows_routed, rows_shared;  // token rows of the routed / shared buffers
 };
 
 struct TileInfo {
@@ -350,7 +352,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r,
         uint32_t v[32];
         tmem_ld_32x32b_x32(tbase + (uint32_t)c0, v);
         tmem_ld_wait();
-        const int nj = min(32, ti.nrows - c0);
+        int nj = min(32, ti.nrows - c0);
+        if (!MOE_CHECK((int64_t)ti.row0 + c0 + nj <= (routed ? p.rows_routed : p.rows_shared)))
+          nj = 0;  // rows outside the buffer: recorded, stores skipped
         if (MODE == kDown) {
           const int col = ti.ft * 128 + frow;
           if (routed && p.routed_f32) {
@@ -527,6 +531,8 @@ cudaError_t launch_grouped_gemms(const Shape& s, const GroupedGemmArgs& a, int n
     p.g_shared = shared ? a.g_shared : nullptr;
     p.u_shared = shared ? a.u_shared : nullptr;
     p.status = status;
+    p.rows_routed = s.cap;
+    p.rows_shared = s.T;
     p.wait_limit_ns = wait_limit_ns;
     // decode: 128-deep stages (two 64-wide sub-tiles) so each weight row is
     // fetched 256 contiguous bytes at a time (measured 4 % faster than 64-deep)
@@ -569,6 +575,8 @@ cudaError_t launch_grouped_gemms(const Shape& s, const GroupedGemmArgs& a, int n
     p.ld_shared = s.d;
     p.shared_f32 = 1;
     p.status = status;
+    p.rows_routed = s.cap;
+    p.rows_shared = s.T;
     p.wait_limit_ns = wait_limit_ns;
     cudaError_t err = small ? launch_one<kDown, 32, 10>(m, p, num_sms, st)
                             : launch_one<kDown, 256, 4>(m, p, num_sms, st);
@@ -578,3 +586,5 @@ cudaError_t launch_grouped_gemms(const Shape& s, const GroupedGemmArgs& a, int n
 }
 
 }  // namespace moe
+
+MOE_CHECKS_UNIT(grouped_gemm)

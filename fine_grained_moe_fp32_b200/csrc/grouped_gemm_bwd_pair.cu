@@ -31,6 +31,7 @@
 #include <cudaTypedefs.h>
 
 #include "moe_internal.h"
+#include "checks.cuh"
 #include "ptx_sm100.cuh"
 
 namespace moe {
@@ -89,6 +90,7 @@ struct PBParams {
   int ucol_routed, ucol_shared;  // dgrad-down: column of dU in the output
   unsigned int* status;
   uint64_t wait_limit_ns;
+  int64_t rows_routed, rows_shared;  // dgrads: token rows of the routed / shared buffers
 };
 
 struct PBTile {
@@ -490,7 +492,9 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
       const float* gsrc = routed ? p.g_routed : p.g_shared;
       const float* usrc = routed ? p.u_routed : p.u_shared;
       const int ldgu = routed ? p.ld_gu_routed : p.ld_gu_shared;
-      const int nj = min(32, t.nrows - c0);
+      int nj = min(32, t.nrows - c0);
+      if (!MOE_CHECK((int64_t)t.row0 + c0 + nj <= (routed ? p.rows_routed : p.rows_shared)))
+        nj = 0;
       const size_t at0 = (size_t)(t.row0 + c0) * ldgu + f0 + mrow;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
@@ -641,7 +645,9 @@ grouped_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
         uint32_t v[32];
         tmem_ld_32x32b_x32(tbase + (uint32_t)c0, v);
         tmem_ld_wait();
-        const int nj = min(32, ncols - c0);
+        int nj = min(32, ncols - c0);
+        if (!MOE_CHECK((int64_t)t.row0 + c0 + nj <= (routed ? p.rows_routed : p.rows_shared)))
+          nj = 0;  // token rows outside the buffer: recorded, stores skipped
         if (MODE == kPDgradDown) {
           // SwiGLU backward on a 32-token x 128-feature tile staged in smem
           uint16_t* out = static_cast<uint16_t*>(routed ? p.out_routed : p.out_shared);
@@ -786,6 +792,8 @@ PBParams pb_base(const Shape& s, const int32_t* offsets, unsigned int* status, u
   p.offsets = offsets;
   p.status = status;
   p.wait_limit_ns = wait_ns;
+  p.rows_routed = s.cap;
+  p.rows_shared = s.T;
   return p;
 }
 
@@ -936,3 +944,5 @@ cudaError_t launch_backward_gemms_pair(const Shape& s, const BackwardGemmArgs& a
 }
 
 }  // namespace moe
+
+MOE_CHECKS_UNIT(grouped_gemm_bwd_pair)

@@ -27,6 +27,7 @@
 #include <cudaTypedefs.h>
 
 #include "moe_internal.h"
+#include "checks.cuh"
 #include "ptx_sm100.cuh"
 
 namespace moe {
@@ -68,6 +69,7 @@ struct PairParams {
   float *g_routed, *u_routed, *g_shared, *u_shared;  // training: fp32 pre-activations
   unsigned int* status;
   uint64_t wait_limit_ns;
+  int64_t rows_routed, rows_shared;  // token rows of the routed / shared buffers
 };
 
 struct PTile {
@@ -367,7 +369,9 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
         uint32_t v[32];
         tmem_ld_32x32b_x32(tbase + (uint32_t)c0, v);
         tmem_ld_wait();
-        const int nj = min(32, t.nrows - c0);
+        int nj = min(32, t.nrows - c0);
+        if (!MOE_CHECK((int64_t)t.row0 + c0 + nj <= (routed ? p.rows_routed : p.rows_shared)))
+          nj = 0;  // rows outside the buffer: recorded, stores skipped
         if (MODE == kPairDown) {
           const int col = t.ft * 256 + (int)rank * 128 + frow;
           if (routed && p.routed_f32) {
@@ -561,6 +565,8 @@ cudaError_t launch_grouped_gemms_pair(const Shape& s, const GroupedGemmArgs& a, 
     p.g_shared = shared ? a.g_shared : nullptr;
     p.u_shared = shared ? a.u_shared : nullptr;
     p.status = status;
+    p.rows_routed = s.cap;
+    p.rows_shared = s.T;
     p.wait_limit_ns = wait_limit_ns;
     if ((err = launch_pair<kPairSwiGLU>(m, p, num_sms, st)) != cudaSuccess) return err;
     if (between != nullptr && (err = cudaEventRecord(between, st)) != cudaSuccess) return err;
@@ -594,6 +600,8 @@ cudaError_t launch_grouped_gemms_pair(const Shape& s, const GroupedGemmArgs& a, 
     p.ld_shared = s.d;
     p.shared_f32 = 1;
     p.status = status;
+    p.rows_routed = s.cap;
+    p.rows_shared = s.T;
     p.wait_limit_ns = wait_limit_ns;
     if ((err = launch_pair<kPairDown>(m, p, num_sms, st)) != cudaSuccess) return err;
   }
@@ -601,3 +609,5 @@ cudaError_t launch_grouped_gemms_pair(const Shape& s, const GroupedGemmArgs& a, 
 }
 
 }  // namespace moe
+
+MOE_CHECKS_UNIT(grouped_gemm_pair)

@@ -4,6 +4,7 @@
 #include <cstring>
 
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 #include <mutex>
 
 #include "../../include/moe_b200.h"
@@ -43,6 +44,27 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
+}  // namespace
+
+cudaError_t checks_init_all(unsigned int* status) {
+#ifdef MOE_CHECKS
+  cudaError_t e;
+  if ((e = checks_init_grouped_gemm(status)) != cudaSuccess ||
+      (e = checks_init_grouped_gemm_pair(status)) != cudaSuccess ||
+      (e = checks_init_grouped_gemm_bwd(status)) != cudaSuccess ||
+      (e = checks_init_grouped_gemm_bwd_pair(status)) != cudaSuccess ||
+      (e = checks_init_permute(status)) != cudaSuccess ||
+      (e = checks_init_combine(status)) != cudaSuccess ||
+      (e = checks_init_backward(status)) != cudaSuccess)
+    return e;
+#else
+  (void)status;
+#endif
+  return cudaSuccess;
+}
+
+namespace {
+
 const DeviceInfo* device_info() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
@@ -54,12 +76,35 @@ const DeviceInfo* device_info() {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
     d.status = static_cast<unsigned int*>(p);
+    if (checks_init_all(d.status) != cudaSuccess) return nullptr;
     d.ready = true;
   }
   return &d;
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Host-side NVTX range around one phase of a call (visible in Nsight
+// timelines; a no-op unless a tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
+// Consecutive phase ranges inside a call: next() closes the open one.
+struct NvtxPhases {
+  bool open = false;
+  void next(const char* name) {
+    if (open) nvtxRangePop();
+    nvtxRangePushA(name);
+    open = true;
+  }
+  ~NvtxPhases() {
+    if (open) nvtxRangePop();
+  }
+};
 
 int check_dims(const moe_dims* dims, Shape* s) {
   if (dims == nullptr) return MOE_ERR_INVALID_ARG;
@@ -78,12 +123,16 @@ int check_dims(const moe_dims* dims, Shape* s) {
 
 size_t al256(size_t b) { return (b + 255) & ~size_t(255); }
 
+// Bytes a workspace region takes: its size rounded up to 256, plus the
+// MOE_CHECKS build's guard zone (kGuardBytes, 0 otherwise).
+size_t region(size_t b) { return al256(b) + kGuardBytes; }
+
 moe_ws_layout make_layout(const Shape& s) {
   moe_ws_layout L{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t at = off;
-    off += al256(bytes);
+    off += region(bytes);
     return at;
   };
   L.route_partials = take(router_partials_bytes(s, kPlanSMs));
@@ -110,7 +159,7 @@ moe_train_layout make_train_layout(const Shape& s) {
   size_t off = L.fwd.total;
   auto take = [&](size_t bytes) {
     const size_t at = off;
-    off += al256(bytes);
+    off += region(bytes);
     return at;
   };
   const size_t SI = (size_t)s.S * s.I;
@@ -159,6 +208,7 @@ const char* moe_status_string(int status) {
     case MOE_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
     case MOE_ERR_CUDA: return "CUDA runtime error";
     case MOE_ERR_TIMEOUT: return "a bounded device wait ran out";
+    case MOE_ERR_BOUNDS: return "a device-side bounds check failed (checks build)";
     default: return "unknown status";
   }
 }
@@ -166,7 +216,7 @@ const char* moe_status_string(int status) {
 size_t moe_route_workspace_size(const moe_dims* dims) {
   Shape s;
   if (check_dims(dims, &s) != MOE_OK) return 0;
-  return al256(router_partials_bytes(s, kPlanSMs));
+  return region(router_partials_bytes(s, kPlanSMs));
 }
 
 int moe_route(const moe_dims* dims, const moe_bf16* x, const float* w_gate, const float* bias,
@@ -191,7 +241,7 @@ int moe_route(const moe_dims* dims, const moe_bf16* x, const float* w_gate, cons
 size_t moe_permute_workspace_size(const moe_dims* dims) {
   Shape s;
   if (check_dims(dims, &s) != MOE_OK) return 0;
-  return al256(permute_scratch_bytes(s));
+  return region(permute_scratch_bytes(s));
 }
 
 int moe_permute(const moe_dims* dims, const int32_t* topk_idx, const moe_bf16* x, int32_t* counts,
@@ -311,12 +361,16 @@ int forward_impl(const moe_dims* dims, const moe_bf16* x, const float* w_gate, c
   uint16_t* h_sh = at<uint16_t>(ws, L.h_shared);
   float* y_sh = at<float>(ws, L.y_shared);
 
+  NvtxRange call(train ? "moe_forward_train" : "moe_forward");
+  NvtxPhases ph;
+  ph.next("router");
   cudaError_t e = phase(0, st);
   if (e == cudaSuccess)
     e = launch_router(s, x, w_gate, bias, probs, idx, wts, at<float>(ws, L.route_partials),
                       kPlanSMs, st);
   if (e == cudaSuccess) e = phase(1, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  ph.next("permute");
   e = launch_permute(s, idx, x, counts, offsets, row_of, tor, x_perm,
                      at<void>(ws, L.permute_scratch), di->status, st);
   if (e == cudaSuccess) e = phase(2, st);
@@ -343,10 +397,12 @@ int forward_impl(const moe_dims* dims, const moe_bf16* x, const float* w_gate, c
     a.g_shared = at<float>(ws, TL.g_shared);
     a.u_shared = at<float>(ws, TL.u_shared);
   }
+  ph.next("grouped_gemms");
   e = launch_grouped_gemms(s, a, di->num_sms, di->status, g_wait_limit_ns, st,
                            g_phase_on ? g_phase_events[3] : nullptr);
   if (e == cudaSuccess) e = phase(4, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  ph.next("combine");
   e = launch_combine(s, y_perm, row_of, wts, s.S > 0 ? y_sh : nullptr, y, st);
   if (e == cudaSuccess) e = phase(5, st);
   return cuda_status(e);
@@ -450,6 +506,9 @@ int backward_impl(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
   m.dw_gate = dw_gate;
   m.dx = dx;
   m.dx_f32 = f32;
+  NvtxRange call("moe_backward");
+  NvtxPhases ph;
+  ph.next("combine_router_bwd");
   cudaError_t e = bwd_phase(0, st);
   if (e == cudaSuccess) e = launch_backward_misc_pre(s, m, st);
   if (e == cudaSuccess) e = bwd_phase(1, st);
@@ -484,9 +543,11 @@ int backward_impl(const moe_dims* dims, const moe_bf16* x, const float* w_gate,
   g.dws3 = dws3;
   g.dws2 = dws2;
   g.dw_f32 = f32;
+  ph.next("grouped_gemms_bwd");
   e = launch_backward_gemms(s, g, di->num_sms, di->status, g_wait_limit_ns, st,
                             g_bwd_phase_on ? &g_phase_events[kFwdEvents + 2] : nullptr);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  ph.next("gate_gemms_unpermute");
   e = launch_backward_misc_post(s, m, st);
   if (e == cudaSuccess) e = bwd_phase(6, st);
   return cuda_status(e);
@@ -550,7 +611,7 @@ extern "C" {
 size_t moe_dense_workspace_size(const moe_dims* dims) {
   Shape s;
   if (dense_shape(dims, &s) != MOE_OK) return 0;
-  return dense_h_offset() + al256((size_t)s.T * s.I * 2);
+  return dense_h_offset() + region((size_t)s.T * s.I * 2);
 }
 
 int moe_dense_swiglu(const moe_dims* dims, const moe_bf16* x, const moe_bf16* w1,
@@ -641,7 +702,7 @@ moe_ep_layout make_ep_layout(const Shape& s, int world, int64_t rcap) {
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t at = off;
-    off += al256(bytes);
+    off += region(bytes);
     return at;
   };
   const int El = s.E / world;
@@ -864,6 +925,7 @@ int moe_get_last_device_status(void* stream) {
     case DEV_BAD_EXPERT_ID: return MOE_ERR_INVALID_ARG;
     case DEV_BAD_EP_LAYOUT: return MOE_ERR_INVALID_ARG;
     case DEV_TIMEOUT: return MOE_ERR_TIMEOUT;
+    case DEV_BOUNDS: return MOE_ERR_BOUNDS;
     default: return MOE_ERR_CUDA;
   }
 }

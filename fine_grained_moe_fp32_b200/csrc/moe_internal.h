@@ -14,7 +14,30 @@ enum DevStatus : unsigned int {
   DEV_BAD_EXPERT_ID = 1,
   DEV_TIMEOUT = 2,
   DEV_BAD_EP_LAYOUT = 3,  // expert-parallel counts inconsistent or over capacity
+  DEV_BOUNDS = 4,         // a MOE_CHECKS bounds check failed (the access was skipped)
 };
+
+// Bytes of the guard zone after every workspace region (and at the end of
+// every workspace) in the MOE_CHECKS build: the library never writes them,
+// so a caller that fills the workspace with a pattern can detect overruns.
+#ifdef MOE_CHECKS
+constexpr size_t kGuardBytes = 256;
+#else
+constexpr size_t kGuardBytes = 0;
+#endif
+
+// MOE_CHECKS build: point every translation unit's copy of the status
+// pointer at the device status word (checks.cuh); a no-op otherwise.
+cudaError_t checks_init_all(unsigned int* status);
+#ifdef MOE_CHECKS
+cudaError_t checks_init_grouped_gemm(unsigned int* status);
+cudaError_t checks_init_grouped_gemm_pair(unsigned int* status);
+cudaError_t checks_init_grouped_gemm_bwd(unsigned int* status);
+cudaError_t checks_init_grouped_gemm_bwd_pair(unsigned int* status);
+cudaError_t checks_init_permute(unsigned int* status);
+cudaError_t checks_init_combine(unsigned int* status);
+cudaError_t checks_init_backward(unsigned int* status);
+#endif
 
 __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 __host__ __device__ inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }

@@ -15,6 +15,7 @@
 // CTA (permute_index_one_chunk_kernel): the same ranks and rows, two launches
 // fewer.
 #include "moe_internal.h"
+#include "checks.cuh"
 
 namespace moe {
 namespace {
@@ -79,7 +80,8 @@ permute_scan_kernel(const int32_t* __restrict__ chunk_counts, int nchunks, int E
   if (e < E) {
     offsets[e] = start;
     if (e == E - 1) offsets[E] = end;
-    for (int r = start + total; r < end; ++r) token_of_row[r] = -1;
+    for (int r = start + total; r < end; ++r)
+      if (MOE_CHECK(r < cap)) token_of_row[r] = -1;
   }
   const int used = scan[E - 1];
   for (int64_t r = used + e; r < cap; r += blockDim.x) token_of_row[r] = -1;
@@ -88,7 +90,8 @@ permute_scan_kernel(const int32_t* __restrict__ chunk_counts, int nchunks, int E
 __global__ void __launch_bounds__(kChunk)
 permute_scatter_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
                        const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ offsets,
-                       int32_t* __restrict__ row_of, int32_t* __restrict__ token_of_row) {
+                       int32_t* __restrict__ row_of, int32_t* __restrict__ token_of_row,
+                       int64_t cap) {
   __shared__ unsigned int masks[kWarps][kMaxE];
   __shared__ int pre[kWarps][kMaxE];
   __shared__ int base[kMaxE];
@@ -126,7 +129,10 @@ permute_scatter_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
       int row = -1;
       if (e >= 0 && e < E && !dup) {
         row = base[e] + pre[warp][e] + __popc(masks[warp][e] & lt);
-        token_of_row[row] = t;
+        if (MOE_CHECK(row >= 0 && row < cap))
+          token_of_row[row] = t;
+        else
+          row = -1;
       }
       row_of[(size_t)t * k + j] = row;
     }
@@ -189,7 +195,8 @@ permute_index_one_chunk_kernel(const int32_t* __restrict__ idx, int T, int k, in
     offsets[t] = start;
     if (t == E - 1) offsets[E] = end;
     base[t] = start;
-    for (int r = start + total; r < end; ++r) token_of_row[r] = -1;
+    for (int r = start + total; r < end; ++r)
+      if (MOE_CHECK(r < cap)) token_of_row[r] = -1;
   }
   const int used = scan[E - 1];
   for (int64_t r = used + t; r < cap; r += blockDim.x) token_of_row[r] = -1;
@@ -203,7 +210,10 @@ permute_index_one_chunk_kernel(const int32_t* __restrict__ idx, int T, int k, in
       int row = -1;
       if (e >= 0 && e < E && !dup) {
         row = base[e] + pre[warp][e] + __popc(masks[warp][e] & lt);
-        token_of_row[row] = t;
+        if (MOE_CHECK(row >= 0 && row < cap))
+          token_of_row[row] = t;
+        else
+          row = -1;
       }
       row_of[(size_t)t * k + j] = row;
     }
@@ -221,6 +231,7 @@ permute_gather_kernel(const uint16_t* __restrict__ x, int T, int d,
   const int lane = threadIdx.x & 31;
   if (r >= cap || r >= offsets[E]) return;
   const int tok = token_of_row[r];
+  (void)MOE_CHECK(tok >= -1 && tok < T);  // a token id no row can hold
   uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)r * d);
   const int nv = d / 8;
   if (tok >= 0 && tok < T) {
@@ -259,7 +270,7 @@ cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16
                                              chunk_base, counts, offsets, token_of_row);
     if (nchunks > 0) {
       permute_scatter_kernel<<<nchunks, kChunk, 0, st>>>(topk_idx, s.T, s.k, s.E, chunk_base,
-                                                         offsets, row_of, token_of_row);
+                                                         offsets, row_of, token_of_row, s.cap);
     }
   }
   if (s.cap > 0 && x_perm != nullptr) {
@@ -271,3 +282,5 @@ cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16
 }
 
 }  // namespace moe
+
+MOE_CHECKS_UNIT(permute)

@@ -59,7 +59,7 @@ extern "C" int moe_route_noalloc(const moe_dims* dims, const moe_bf16* x, const 
     // invalid or unsupported dims: let moe_route report which
     return moe_route(dims, x, w_gate, bias, probs, topk_idx, topk_w, nullptr, 0, stream);
   }
-  if (moe_route_workspace_size(dims) > moe::kScratchBytes) return MOE_ERR_WORKSPACE;
+  if (moe_route_workspace_size(dims) - moe::kGuardBytes > moe::kScratchBytes) return MOE_ERR_WORKSPACE;
   void* scratch = moe::scratch_on_current_device();
   if (scratch == nullptr) return MOE_ERR_CUDA;
   return moe_route(dims, x, w_gate, bias, probs, topk_idx, topk_w, scratch, moe::kScratchBytes,

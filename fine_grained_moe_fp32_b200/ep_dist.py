@@ -95,7 +95,8 @@ class EPGroup:
         self.ws1, self.ws3, self.ws2 = to(inputs["ws1"]), to(inputs["ws3"]), to(inputs["ws2"])
         self.dm = M.dims(T, cfg.d, cfg.E, cfg.k, cfg.I, cfg.S, align)
         self.recv_cap = M.ep_recv_capacity(self.dm, self.world)
-        self.ws = M.alloc_workspace(M.ep_workspace_size(self.dm, self.world), self.device)
+        self.ws = M.guard_layout(M.alloc_workspace(M.ep_workspace_size(self.dm, self.world),
+                                                   self.device), M.ep_layout(self.dm, self.world))
         self.views = M.ep_workspace_views(self.dm, self.world, self.ws)
         bf = dict(dtype=torch.bfloat16, device=self.device)
         self.x_recv = torch.empty((self.recv_cap, cfg.d), **bf)

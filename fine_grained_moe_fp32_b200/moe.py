@@ -12,7 +12,12 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
+# MOE_CHECKS=1 in the environment selects the bounds-checking build of the
+# library (device bounds checks recorded as MOE_ERR_BOUNDS, a guard zone
+# after every workspace region); it is built by `build --checks`.
+CHECKS = os.environ.get("MOE_CHECKS", "0") not in ("", "0")
+LIB_PATH = os.path.join(_PKG, "libmoe_b200_checks.so" if CHECKS else "libmoe_b200.so")
+GUARD_BYTES = 256 if CHECKS else 0
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = -1
@@ -20,6 +25,7 @@ MOE_ERR_UNSUPPORTED_SHAPE = -2
 MOE_ERR_WORKSPACE = -3
 MOE_ERR_CUDA = -4
 MOE_ERR_TIMEOUT = -5
+MOE_ERR_BOUNDS = -6
 
 # every symbol declared in include/moe_b200.h
 EXPORTED = (
@@ -191,9 +197,62 @@ def forward_layout(dm: MoeDims) -> dict:
     return {n: getattr(L, n) for n, _ in MoeWsLayout._fields_}
 
 
+CANARY = 0xA5  # checks build: the byte every workspace starts filled with
+_guarded = []  # checks build: (weak reference to a workspace, [(start, end) guard bytes])
+
+
 def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
-    """A uint8 device buffer of at least nbytes (torch's allocator aligns to 512 B)."""
-    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+    """A uint8 device buffer of at least nbytes (torch's allocator aligns to 512 B).
+    Checks build: filled with CANARY (so a region read before it is written
+    shows up as a parity failure) and registered with its trailing guard
+    zone, which the library never writes."""
+    ws = torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+    if CHECKS:
+        import weakref
+        ws.fill_(CANARY)
+        n = int(nbytes)
+        _guarded.append((weakref.ref(ws), [(n - GUARD_BYTES, n)] if n >= GUARD_BYTES else []))
+    return ws
+
+
+def guard_layout(ws: torch.Tensor, layout: dict) -> torch.Tensor:
+    """Checks build: register the guard zone in front of every region of a
+    workspace layout (the 256 bytes before each offset: the previous
+    region's guard).  A no-op otherwise."""
+    if CHECKS:
+        import weakref
+        offs = sorted({v for k, v in _flatten(layout).items() if v > 0})
+        _guarded.append((weakref.ref(ws), [(o - GUARD_BYTES, o) for o in offs]))
+    return ws
+
+
+def _flatten(layout: dict) -> dict:
+    out = {}
+    for k, v in layout.items():
+        if isinstance(v, dict):
+            out.update({f"{k}.{kk}": vv for kk, vv in _flatten(v).items()})
+        else:
+            out[k] = int(v)
+    return out
+
+
+def check_guards() -> list:
+    """Checks build: every registered guard zone of every live workspace
+    still holds CANARY.  Returns a list of (workspace bytes, start, end) that
+    do not (empty when all are intact); forgets workspaces that are gone."""
+    bad, keep = [], []
+    for ref, ranges in _guarded:
+        ws = ref()
+        if ws is None:
+            continue
+        keep.append((ref, ranges))
+        for a, b in ranges:
+            if a < 0 or b > ws.numel():
+                bad.append((ws.numel(), a, b))
+            elif not bool((ws[a:b] == CANARY).all()):
+                bad.append((ws.numel(), a, b))
+    _guarded[:] = keep
+    return bad
 
 
 # ------------------------------------------------------------------ calls
@@ -518,7 +577,8 @@ class EPRanks:
         self.dm = dims(T, cfg.d, cfg.E, cfg.k, cfg.I, cfg.S, align)
         self.recv_cap = ep_recv_capacity(self.dm, world)
         nbytes = ep_workspace_size(self.dm, world)
-        self.ws = [alloc_workspace(nbytes, self.device) for _ in range(world)]
+        self.ws = [guard_layout(alloc_workspace(nbytes, self.device), ep_layout(self.dm, world))
+                   for _ in range(world)]
         bf = dict(dtype=torch.bfloat16, device=self.device)
         self.x_recv = [torch.empty((self.recv_cap, cfg.d), **bf) for _ in range(world)]
         self.y_recv = [torch.empty((self.recv_cap, cfg.d), dtype=torch.float32, device=self.device)
@@ -702,13 +762,16 @@ class MoELayer:
 
     def workspace(self, T: int) -> torch.Tensor:
         if self._ws is None or self._ws_T != T:
-            self._ws = alloc_workspace(workspace_size(self.dims(T)), self.device)
+            self._ws = guard_layout(alloc_workspace(workspace_size(self.dims(T)), self.device),
+                                    forward_layout(self.dims(T)))
             self._ws_T = T
         return self._ws
 
     def train_workspace(self, T: int) -> torch.Tensor:
         if getattr(self, "_tws", None) is None or self._tws_T != T:
-            self._tws = alloc_workspace(train_workspace_size(self.dims(T)), self.device)
+            self._tws = guard_layout(
+                alloc_workspace(train_workspace_size(self.dims(T)), self.device),
+                train_layout(self.dims(T)))
             self._tws_T = T
         return self._tws
 

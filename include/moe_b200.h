@@ -54,7 +54,9 @@ enum {
   MOE_ERR_UNSUPPORTED_SHAPE = -2, /* shape outside the limits above       */
   MOE_ERR_WORKSPACE = -3,         /* workspace missing, small or unaligned */
   MOE_ERR_CUDA = -4,              /* a CUDA runtime call failed            */
-  MOE_ERR_TIMEOUT = -5            /* a bounded device-side wait ran out    */
+  MOE_ERR_TIMEOUT = -5,           /* a bounded device-side wait ran out    */
+  MOE_ERR_BOUNDS = -6             /* a device bounds check failed (only the
+                                     MOE_CHECKS build checks; see below)  */
 };
 
 /* Layer dimensions.

@@ -24,3 +24,21 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _checks_build_guards(request):
+    """With MOE_CHECKS=1 (the bounds-checking build of the library): after
+    every GPU test, no device bounds check may have failed and every guard
+    zone of every live workspace must still hold its canary bytes."""
+    yield
+    if "gpu" not in request.node.keywords:
+        return
+    from fine_grained_moe_fp32_b200 import moe as M
+    if not M.CHECKS:
+        return
+    import torch
+    torch.cuda.synchronize()
+    assert M.device_status() != M.MOE_ERR_BOUNDS, "a device bounds check failed"
+    bad = M.check_guards()
+    assert not bad, f"guard zones overwritten: {bad[:8]}"

@@ -178,7 +178,7 @@ def test_ipc_calls_rejected_on_host(lib):
 
 
 def test_status_strings(lib):
-    for s in (0, -1, -2, -3, -4, -5):
+    for s in (0, -1, -2, -3, -4, -5, -6):
         assert M.status_string(s) != "unknown status"
 
 
@@ -193,3 +193,24 @@ def test_no_alloc_route_rejects_shapes_beyond_its_scratch(lib):
                                  None) == M.MOE_ERR_WORKSPACE
     assert M.route_workspace_size(M.dims(T=32768, d=5120, E=128, k=6, I=1408, n_shared=2,
                                          align=16)) <= (16 << 20)
+
+
+def test_guard_zone_bookkeeping(monkeypatch):
+    """The checks build's canary bookkeeping (host side, on a CPU tensor): a
+    fresh workspace holds the canary everywhere; writing into a region leaves
+    its guards intact; writing into a guard zone is reported."""
+    monkeypatch.setattr(M, "CHECKS", True)
+    monkeypatch.setattr(M, "GUARD_BYTES", 256)
+    monkeypatch.setattr(M, "_guarded", [])
+    layout = {"a": 0, "b": 1024, "c": 2048, "total": 4096}
+    ws = M.guard_layout(M.alloc_workspace(4096, "cpu"), layout)
+    assert bool((ws == M.CANARY).all())
+    ws[0:700] = 1                     # region a (its guard is [768, 1024))
+    ws[1024:1700] = 2                 # region b
+    assert M.check_guards() == []
+    ws[1800] = 0                      # region b's guard
+    ws[4095] = 0                      # the trailing guard
+    bad = M.check_guards()
+    assert (4096, 1792, 2048) in bad and (4096, 3840, 4096) in bad
+    del ws
+    assert M.check_guards() == []     # a freed workspace is forgotten

@@ -89,3 +89,32 @@ def test_forward_captures_into_a_cuda_graph(name, T):
     torch.cuda.synchronize()
     assert M.device_status() == M.MOE_OK
     assert torch.equal(y.view(torch.int16), layer(x2).view(torch.int16))
+
+
+def test_out_of_range_row_is_skipped_and_flagged_by_the_checks_build():
+    """moe_combine given a row index past the permuted buffer for one pair:
+    that pair contributes nothing in both builds (the kernel's own range
+    test skips it); the MOE_CHECKS build also records MOE_ERR_BOUNDS, the
+    normal build records nothing.  Every other token is unaffected."""
+    T, d, E, k = 8, 256, 16, 2
+    dm = M.dims(T, d, E, k, 64, 0, 16)
+    cap = M.capacity(dm)
+    gen = torch.Generator().manual_seed(9)
+    y_perm = torch.randn((cap, d), generator=gen).cuda()
+    rows = torch.arange(T * k, dtype=torch.int32)
+    w = torch.full((T, k), 0.5)
+    bad = rows.clone()
+    bad[3] = cap + 5                  # token 1, slot 1
+    y = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    y_ok = torch.empty_like(y)
+    M.combine(dm, y_perm, rows.cuda(), w.cuda(), None, y_ok)
+    torch.cuda.synchronize()
+    assert M.device_status() == M.MOE_OK
+    M.combine(dm, y_perm, bad.cuda(), w.cuda(), None, y)
+    status = M.device_status()
+    assert status == (M.MOE_ERR_BOUNDS if M.CHECKS else M.MOE_OK)
+    assert M.device_status() == M.MOE_OK        # cleared by the read
+    keep = [t for t in range(T) if t != 1]
+    assert torch.equal(y[keep].view(torch.int16), y_ok[keep].view(torch.int16))
+    want = (0.5 * y_perm[2].float()).to(torch.bfloat16)   # token 1's first slot alone
+    assert torch.equal(y[1].view(torch.int16), want.view(torch.int16))
