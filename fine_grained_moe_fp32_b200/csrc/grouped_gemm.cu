@@ -483,12 +483,19 @@ cudaError_t launch_one(const CUtensorMap* maps, const GemmParams& p, int num_sms
 
 }  // namespace
 
+bool uses_pair_gemms(const Shape& s) {
+  return (int64_t)s.T * s.k > (int64_t)24 * s.E && pair_gemms_supported(s);
+}
+
 cudaError_t launch_grouped_gemms(const Shape& s, const GroupedGemmArgs& a, int num_sms,
                                  unsigned int* status, uint64_t wait_limit_ns, cudaStream_t st,
                                  cudaEvent_t between) {
-  const bool shared = s.S > 0 && a.x != nullptr && a.ws1 != nullptr && a.ws3 != nullptr &&
-                      a.ws2 != nullptr && a.h_shared != nullptr && a.y_shared != nullptr &&
-                      s.T > 0;
+  const bool shared = a.part != GroupedGemmArgs::kRoutedOnly && s.S > 0 && a.x != nullptr &&
+                      a.ws1 != nullptr && a.ws3 != nullptr && a.ws2 != nullptr &&
+                      a.h_shared != nullptr && a.y_shared != nullptr && s.T > 0;
+  // routed groups in the schedule (none for a shared-only launch; the routed
+  // maps stay valid, they are just not used)
+  const int E_run = a.part == GroupedGemmArgs::kSharedOnly ? 0 : s.E;
   const bool small = (int64_t)s.T * s.k <= (int64_t)24 * s.E;  // decode-sized segments
   if (!small && pair_gemms_supported(s))
     return launch_grouped_gemms_pair(s, a, num_sms, status, wait_limit_ns, st, between);
@@ -510,7 +517,7 @@ cudaError_t launch_grouped_gemms(const Shape& s, const GroupedGemmArgs& a, int n
     }
     if (!ok) return cudaErrorInvalidValue;
     GemmParams p{};
-    p.E = s.E;
+    p.E = E_run;
     p.has_shared = shared ? 1 : 0;
     p.T = s.T;
     p.ft_routed = s.I / 64;
@@ -557,7 +564,7 @@ cudaError_t launch_grouped_gemms(const Shape& s, const GroupedGemmArgs& a, int n
     }
     if (!ok) return cudaErrorInvalidValue;
     GemmParams p{};
-    p.E = s.E;
+    p.E = E_run;
     p.has_shared = shared ? 1 : 0;
     p.T = s.T;
     p.ft_routed = s.d / 128;

@@ -529,9 +529,12 @@ bool pair_gemms_supported(const Shape& s) { return s.I % 128 == 0 && s.d % 256 =
 cudaError_t launch_grouped_gemms_pair(const Shape& s, const GroupedGemmArgs& a, int num_sms,
                                       unsigned int* status, uint64_t wait_limit_ns,
                                       cudaStream_t st, cudaEvent_t between) {
-  const bool shared = s.S > 0 && a.x != nullptr && a.ws1 != nullptr && a.ws3 != nullptr &&
-                      a.ws2 != nullptr && a.h_shared != nullptr && a.y_shared != nullptr &&
-                      s.T > 0;
+  const bool shared = a.part != GroupedGemmArgs::kRoutedOnly && s.S > 0 && a.x != nullptr &&
+                      a.ws1 != nullptr && a.ws3 != nullptr && a.ws2 != nullptr &&
+                      a.h_shared != nullptr && a.y_shared != nullptr && s.T > 0;
+  // routed groups in the schedule (none for a shared-only launch; the routed
+  // maps stay valid, they are just not used)
+  const int E_run = a.part == GroupedGemmArgs::kSharedOnly ? 0 : s.E;
   const int SI = s.S * s.I;
   CUtensorMap m[6];
   cudaError_t err;
@@ -547,7 +550,7 @@ cudaError_t launch_grouped_gemms_pair(const Shape& s, const GroupedGemmArgs& a, 
       m[3] = m[0], m[4] = m[1], m[5] = m[2];
     if (!ok) return cudaErrorInvalidValue;
     PairParams p{};
-    p.E = s.E;
+    p.E = E_run;
     p.has_shared = shared ? 1 : 0;
     p.T = s.T;
     p.ft_routed = s.I / 128;
@@ -584,7 +587,7 @@ cudaError_t launch_grouped_gemms_pair(const Shape& s, const GroupedGemmArgs& a, 
     m[4] = m[3];
     if (!ok) return cudaErrorInvalidValue;
     PairParams p{};
-    p.E = s.E;
+    p.E = E_run;
     p.has_shared = shared ? 1 : 0;
     p.T = s.T;
     p.ft_routed = p.ft_shared = s.d / 256;

@@ -40,9 +40,14 @@ struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
   unsigned int* status = nullptr;
+  // prefill forward: the shared experts' GEMMs run on `side` while the
+  // router and the permutation run on the caller's stream (fork, join)
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
+std::mutex g_fork_mu;  // one fork/join sequence at a time (the events are per device)
 
 }  // namespace
 
@@ -77,6 +82,10 @@ const DeviceInfo* device_info() {
     if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
     d.status = static_cast<unsigned int*>(p);
     if (checks_init_all(d.status) != cudaSuccess) return nullptr;
+    if (cudaStreamCreateWithFlags(&d.side, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&d.join, cudaEventDisableTiming) != cudaSuccess)
+      return nullptr;
     d.ready = true;
   }
   return &d;
@@ -361,20 +370,6 @@ int forward_impl(const moe_dims* dims, const moe_bf16* x, const float* w_gate, c
   uint16_t* h_sh = at<uint16_t>(ws, L.h_shared);
   float* y_sh = at<float>(ws, L.y_shared);
 
-  NvtxRange call(train ? "moe_forward_train" : "moe_forward");
-  NvtxPhases ph;
-  ph.next("router");
-  cudaError_t e = phase(0, st);
-  if (e == cudaSuccess)
-    e = launch_router(s, x, w_gate, bias, probs, idx, wts, at<float>(ws, L.route_partials),
-                      kPlanSMs, st);
-  if (e == cudaSuccess) e = phase(1, st);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
-  ph.next("permute");
-  e = launch_permute(s, idx, x, counts, offsets, row_of, tor, x_perm,
-                     at<void>(ws, L.permute_scratch), di->status, st);
-  if (e == cudaSuccess) e = phase(2, st);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
   GroupedGemmArgs a{};
   a.x_perm = x_perm;
   a.offsets = offsets;
@@ -397,11 +392,49 @@ int forward_impl(const moe_dims* dims, const moe_bf16* x, const float* w_gate, c
     a.g_shared = at<float>(ws, TL.g_shared);
     a.u_shared = at<float>(ws, TL.u_shared);
   }
+  // Prefill-sized batches: the shared experts' GEMMs do not depend on the
+  // routing.  After the router they go to the side stream, launched before
+  // the permutation so their CTAs are resident first: the permutation's
+  // HBM-bound gather then runs on the SMs beside those compute-bound GEMMs.
+  // The caller's stream waits for them before the combine.  Measured on the
+  // same box against one stream: 2.6 % faster at T = 4096, 1.3 % at 16384;
+  // the training forward (which also stores g and u) was 1.2 % slower, so
+  // it keeps one stream.
+  const bool split = !train && s.S > 0 && s.T > 0 && uses_pair_gemms(s);
+  std::unique_lock<std::mutex> fork_lock(g_fork_mu, std::defer_lock);
+  NvtxRange call(train ? "moe_forward_train" : "moe_forward");
+  NvtxPhases ph;
+  ph.next("router");
+  cudaError_t e = phase(0, st);
+  if (e == cudaSuccess)
+    e = launch_router(s, x, w_gate, bias, probs, idx, wts, at<float>(ws, L.route_partials),
+                      kPlanSMs, st);
+  if (e == cudaSuccess) e = phase(1, st);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (split) {
+    ph.next("shared_experts (side stream)");
+    fork_lock.lock();
+    GroupedGemmArgs sh = a;
+    sh.part = GroupedGemmArgs::kSharedOnly;
+    if ((e = cudaEventRecord(di->fork, st)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(di->side, di->fork, 0)) != cudaSuccess ||
+        (e = launch_grouped_gemms(s, sh, di->num_sms, di->status, g_wait_limit_ns, di->side)) !=
+            cudaSuccess ||
+        (e = cudaEventRecord(di->join, di->side)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    a.part = GroupedGemmArgs::kRoutedOnly;
+  }
+  ph.next("permute");
+  e = launch_permute(s, idx, x, counts, offsets, row_of, tor, x_perm,
+                     at<void>(ws, L.permute_scratch), di->status, st);
+  if (e == cudaSuccess) e = phase(2, st);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
   ph.next("grouped_gemms");
   e = launch_grouped_gemms(s, a, di->num_sms, di->status, g_wait_limit_ns, st,
                            g_phase_on ? g_phase_events[3] : nullptr);
   if (e == cudaSuccess) e = phase(4, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (split && (e = cudaStreamWaitEvent(st, di->join, 0)) != cudaSuccess) return MOE_ERR_CUDA;
   ph.next("combine");
   e = launch_combine(s, y_perm, row_of, wts, s.S > 0 ? y_sh : nullptr, y, st);
   if (e == cudaSuccess) e = phase(5, st);

@@ -73,6 +73,11 @@ struct GroupedGemmArgs {
   uint16_t* h_perm;  // [cap, I]
   void* y_perm;      // [cap, d] fp32, or bf16 when !y_perm_f32 (the dense FFN's y)
   bool y_perm_f32 = true;
+  // which groups a launch covers: both, the routed experts only, or the
+  // shared experts only (the shared ones do not depend on the routing, so
+  // they can run while the router and the permutation do)
+  enum Part : int { kAll = 0, kRoutedOnly = 1, kSharedOnly = 2 };
+  int part = kAll;
   // shared experts (S > 0 and all non-null to enable)
   const uint16_t* x;  // [T, d]
   const uint16_t *ws1, *ws3, *ws2;
@@ -88,6 +93,10 @@ struct GroupedGemmArgs {
 cudaError_t launch_grouped_gemms(const Shape& s, const GroupedGemmArgs& a, int num_sms,
                                  unsigned int* status, uint64_t wait_limit_ns, cudaStream_t st,
                                  cudaEvent_t between = nullptr);
+
+// true when launch_grouped_gemms runs the paired-CTA kernels (prefill-sized
+// segments) for this shape
+bool uses_pair_gemms(const Shape& s);
 
 // ---- paired-CTA grouped GEMMs for prefill-sized segments (grouped_gemm_pair.cu)
 bool pair_gemms_supported(const Shape& s);

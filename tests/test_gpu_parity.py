@@ -365,3 +365,39 @@ def test_forward_full_size_every_segment(cfg):
         y_ref += hg @ w2.T
         y_abs += np.abs(hg) @ np.abs(w2).T
     PU.check_fp32_sum(v["y_shared"], y_ref, y_abs, "y_shared")
+
+
+@pytest.mark.parametrize("cfg,T", [(small_config(T=700, d=512, E=16, k=4, I=256), None),
+                                   (PREFILL_BALANCED, None)],
+                         ids=["pair_prefill_T700", "prefill_balanced"])
+def test_fused_prefill_forward_equals_the_step_calls(cfg, T):
+    """At prefill sizes moe_forward runs the shared experts' GEMMs on a side
+    stream beside the permutation and launches the routed GEMMs alone; the
+    result must be bit-identical to the public step calls (moe_route,
+    moe_permute, moe_grouped_swiglu, moe_combine) on the same batch, whose
+    grouped-GEMM call runs the routed experts in one launch per projection.
+    The combine is fed the fused call's fp32 shared output."""
+    inp = make_inputs(cfg, T=T, device=DEV)
+    g = _gpu(inp)
+    layer = M.MoELayer(g)
+    y = layer(g["x"]).clone()
+    torch.cuda.synchronize()
+    assert M.device_status() == M.MOE_OK
+    dm = M.dims_of(cfg, T=inp["T"])
+    v = M.workspace_views(dm, layer.workspace(inp["T"]))
+    probs, idx, w = _route(dm, g)
+    pm = _permute(dm, idx, g["x"])
+    h, yp = _grouped(dm, pm["x_perm"], pm["offsets"], g)
+    y2 = torch.empty_like(y)
+    M.combine(dm, yp, pm["row_of"], w, v["y_shared"], y2)
+    torch.cuda.synchronize()
+    assert M.device_status() == M.MOE_OK
+    eq = lambda a, b: torch.equal(a.view(torch.int32) if a.dtype == torch.float32 else a.view(torch.int16),  # noqa: E731
+                                  b.view(torch.int32) if b.dtype == torch.float32 else b.view(torch.int16))
+    assert eq(probs, v["probs"]) and torch.equal(idx, v["topk_idx"]) and eq(w, v["topk_w"])
+    for name in ("counts", "offsets", "row_of"):
+        assert torch.equal(pm[name], v[name]), name
+    used = int(pm["offsets"][-1])
+    assert eq(pm["x_perm"][:used], v["x_perm"][:used])
+    assert eq(h[:used], v["h_perm"][:used]) and eq(yp[:used], v["y_perm"][:used])
+    assert eq(y2, y)
