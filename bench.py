@@ -40,8 +40,8 @@ METRIC = "MoE-layer tokens/s (bf16, d=5120, 128E top-6 + 2 shared) and % of roof
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 def forward_kernels(T: int) -> int:
     """Launches of one moe_forward: router GEMM + top-k, the permutation (one
-    index kernel + gather for a batch of at most 256 tokens, else count, scan,
-    scatter + gather), the two grouped GEMMs, the combine."""
+    index kernel + row copy for a batch of at most 256 tokens, else count,
+    scan, scatter + row copy), the two grouped GEMMs, the combine."""
     return 2 + (2 if T <= 256 else 4) + 2 + 1
 BWD_KERNELS = 11      # combine/router bwd (3), 4 grouped GEMMs (dW1 and dW3 in one), 2 gate GEMMs + split sum, un-permute
 BALANCE_KERNELS = 4   # balance partial sums, per-sequence f/P, loss, bias step

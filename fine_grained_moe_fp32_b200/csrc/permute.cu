@@ -8,8 +8,9 @@
 //   permute_scatter_kernel  per chunk: rank of each pair among the chunk's
 //                           earlier tokens of the same expert (warp ballot
 //                           masks + per-warp prefix), row_of / token_of_row
-//   permute_gather_kernel   one warp per row: x_perm[r] = x[token_of_row[r]]
-//                           (zero for padding rows), 16-byte vectors
+//   permute_copy_kernel     one CTA per token: x[t] read once, stored into
+//                           the rows of its k pairs; one CTA per expert zeroes
+//                           its segment's padding rows (16-byte vectors)
 //
 // A batch of at most one chunk (decode) runs count, scan and scatter as one
 // CTA (permute_index_one_chunk_kernel): the same ranks and rows, two launches
@@ -220,26 +221,42 @@ permute_index_one_chunk_kernel(const int32_t* __restrict__ idx, int T, int k, in
   }
 }
 
-constexpr int kGatherWarps = 8;
+constexpr int kCopyThreads = 128;
+constexpr int kMaxK = 8;
 
-__global__ void __launch_bounds__(kGatherWarps * 32)
-permute_gather_kernel(const uint16_t* __restrict__ x, int T, int d,
-                      const int32_t* __restrict__ offsets,
-                      int E, const int32_t* __restrict__ token_of_row, int64_t cap,
-                      uint16_t* __restrict__ x_perm) {
-  const int64_t r = (int64_t)blockIdx.x * kGatherWarps + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (r >= cap || r >= offsets[E]) return;
-  const int tok = token_of_row[r];
-  (void)MOE_CHECK(tok >= -1 && tok < T);  // a token id no row can hold
-  uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)r * d);
+// x_perm, token-major: CTA t < T reads token t's row once and stores it into
+// the rows of its k pairs (row_of); CTA T + e zeroes the padding rows of
+// segment e (the rows between its count and the next segment).  Each x row is
+// read once instead of once per pair, which matters when x does not fit in L2.
+__global__ void __launch_bounds__(kCopyThreads)
+permute_copy_kernel(const uint16_t* __restrict__ x, int T, int d, int k, int E,
+                    const int32_t* __restrict__ row_of, const int32_t* __restrict__ counts,
+                    const int32_t* __restrict__ offsets, int64_t cap,
+                    uint16_t* __restrict__ x_perm) {
   const int nv = d / 8;
-  if (tok >= 0 && tok < T) {
-    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)tok * d);
-    for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
-  } else {
+  if ((int)blockIdx.x >= T) {
+    const int e = (int)blockIdx.x - T;
+    const int64_t r0 = (int64_t)offsets[e] + counts[e], r1 = offsets[e + 1];
+    if (!MOE_CHECK(r0 >= 0 && r1 <= cap)) return;
+    uint4* base = reinterpret_cast<uint4*>(x_perm);
     const uint4 z = make_uint4(0, 0, 0, 0);
-    for (int v = lane; v < nv; v += 32) dst[v] = z;
+    for (int64_t i = r0 * nv + threadIdx.x; i < r1 * nv; i += kCopyThreads) base[i] = z;
+    return;
+  }
+  const int t = blockIdx.x;
+  __shared__ uint4* dst[kMaxK];
+  if ((int)threadIdx.x < k) {
+    const int r = row_of[(size_t)t * k + threadIdx.x];
+    const bool ok = MOE_CHECK(r >= -1 && r < cap) && r >= 0 && r < cap;  // -1: pair skipped
+    dst[threadIdx.x] = ok ? reinterpret_cast<uint4*>(x_perm + (size_t)r * d) : nullptr;
+  }
+  __syncthreads();
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+  for (int v = threadIdx.x; v < nv; v += kCopyThreads) {
+    const uint4 val = __ldg(src + v);
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (j < k && dst[j] != nullptr) dst[j][v] = val;
   }
 }
 
@@ -273,10 +290,9 @@ cudaError_t launch_permute(const Shape& s, const int32_t* topk_idx, const uint16
                                                          offsets, row_of, token_of_row, s.cap);
     }
   }
-  if (s.cap > 0 && x_perm != nullptr) {
-    const unsigned blocks = (unsigned)ceil_div(s.cap, kGatherWarps);
-    permute_gather_kernel<<<blocks, kGatherWarps * 32, 0, st>>>(x, s.T, s.d, offsets, s.E,
-                                                                token_of_row, s.cap, x_perm);
+  if (s.cap > 0 && x_perm != nullptr && s.T + s.E > 0) {
+    permute_copy_kernel<<<(unsigned)(s.T + s.E), kCopyThreads, 0, st>>>(
+        x, s.T, s.d, s.k, s.E, row_of, counts, offsets, s.cap, x_perm);
   }
   return cudaGetLastError();
 }
