@@ -585,7 +585,7 @@ cudaError_t launch_grouped_gemms(const Shape& s, const GroupedGemmArgs& a, int n
     p.rows_routed = s.cap;
     p.rows_shared = s.T;
     p.wait_limit_ns = wait_limit_ns;
-    cudaError_t err = small ? launch_one<kDown, 32, 10>(m, p, num_sms, st)
+    cudaError_t err = small ? launch_one<kDown, 32, 5, 2>(m, p, num_sms, st)
                             : launch_one<kDown, 256, 4>(m, p, num_sms, st);
     if (err != cudaSuccess) return err;
   }
