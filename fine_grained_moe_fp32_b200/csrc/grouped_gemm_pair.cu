@@ -70,10 +70,15 @@ struct PairParams {
   unsigned int* status;
   uint64_t wait_limit_ns;
   int64_t rows_routed, rows_shared;  // token rows of the routed / shared buffers
+  // down GEMM split over K (ksplit > 1): tile (.., ks) sums K chunks
+  // [ks*kit_split, ..) and stores fp32 partials to out_split[ks][row][col]
+  int ksplit, kit_split;
+  float* out_split;
 };
 
 struct PTile {
   int g, ft, row0, nrows, nmma, kit;
+  int ks, k0;  // split of K (down GEMM with ksplit > 1) and its first K chunk
 };
 
 struct PCtl {
@@ -101,13 +106,18 @@ __device__ __forceinline__ PTile pdecode(const PCtl& c, const PairParams& p, int
   t.g = lo;
   const bool routed = lo < p.E;
   const int nft = routed ? p.ft_routed : p.ft_shared;
+  const int nks = p.ksplit > 1 ? p.ksplit : 1;
   const int local = tile - c.prefix[lo];
-  const int tt = local / nft;
-  t.ft = local - tt * nft;
+  t.ks = local % nks;
+  const int rest = local / nks;
+  const int tt = rest / nft;
+  t.ft = rest - tt * nft;
   t.row0 = c.row0[lo] + tt * kNT;
   t.nrows = min(kNT, c.rows[lo] - tt * kNT);
   t.nmma = (t.nrows + 15) & ~15;
-  t.kit = routed ? p.kit_routed : p.kit_shared;
+  const int kit = routed ? p.kit_routed : p.kit_shared;
+  t.k0 = nks > 1 ? t.ks * p.kit_split : 0;
+  t.kit = nks > 1 ? min(p.kit_split, kit - t.k0) : kit;
   return t;
 }
 
@@ -171,7 +181,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
         if (nr < 0) nr = 0;
         ctl.row0[g] = r0;
         ctl.rows[g] = nr;
-        tiles = (int)ceil_div(nr, kNT) * nft;
+        tiles = (int)ceil_div(nr, kNT) * nft * (p.ksplit > 1 ? p.ksplit : 1);
       }
       local[i] = tiles;
       sum += tiles;
@@ -262,7 +272,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
             armed |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           }
-          const int kk = kc * kBK;
+          const int kk = (t.k0 + kc) * kBK;
           const uint32_t sA = sbase + stage * (kABytes + kBBytes);
           const uint32_t sB = sA + kABytes;
           for (int j = 0; j < 2; ++j) {  // the two 64-wide K sub-tiles
@@ -374,7 +384,12 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
           nj = 0;  // rows outside the buffer: recorded, stores skipped
         if (MODE == kPairDown) {
           const int col = t.ft * 256 + (int)rank * 128 + frow;
-          if (routed && p.routed_f32) {
+          if (routed && p.ksplit > 1) {  // one K split's fp32 partial
+            float* out = p.out_split + (size_t)t.ks * p.rows_routed * p.ld_routed;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nj) out[(size_t)(t.row0 + c0 + j) * p.ld_routed + col] = __uint_as_float(v[j]);
+          } else if (routed && p.routed_f32) {
             float* out = static_cast<float*>(p.out_routed);
 #pragma unroll
             for (int j = 0; j < 32; ++j)
@@ -526,6 +541,48 @@ cudaError_t launch_pair(const CUtensorMap* m, const PairParams& p, int num_sms, 
 
 bool pair_gemms_supported(const Shape& s) { return s.I % 128 == 0 && s.d % 256 == 0; }
 
+namespace {
+
+// y[i] = bf16(sum over the K splits of part[s][i]), s ascending, fp32 sum.
+__global__ void split_sum_kernel(const float* __restrict__ part, int splits, int64_t n4,
+                                 uint16_t* __restrict__ y) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  float4 acc = reinterpret_cast<const float4*>(part)[i];
+  for (int sp = 1; sp < splits; ++sp) {
+    const float4 v = reinterpret_cast<const float4*>(part + (size_t)sp * n4 * 4)[i];
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
+  }
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+  reinterpret_cast<uint2*>(y)[i] = make_uint2(*reinterpret_cast<const uint32_t*>(&lo),
+                                              *reinterpret_cast<const uint32_t*>(&hi));
+}
+
+}  // namespace
+
+int down_k_splits(const Shape& s, int num_sms) {
+  if (!uses_pair_gemms(s) || s.S > 0 || s.E != 1) return 1;
+  const int pairs = num_sms / 2;
+  const int base = (int)ceil_div(s.T, kNT) * (s.d / 256);
+  const int kit = s.I / kBK;
+  if (base >= pairs || kit < 4) return 1;
+  // fewest splits among those with the least (waves x K chunks per tile)
+  int best = 1;
+  int64_t best_cost = ceil_div(base, pairs) * kit;
+  for (int sp = 2; sp <= 8 && sp <= kit / 2; ++sp) {
+    const int64_t cost = ceil_div((int64_t)base * sp, pairs) * ceil_div(kit, sp);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = sp;
+    }
+  }
+  return best;
+}
+
 cudaError_t launch_grouped_gemms_pair(const Shape& s, const GroupedGemmArgs& a, int num_sms,
                                       unsigned int* status, uint64_t wait_limit_ns,
                                       cudaStream_t st, cudaEvent_t between) {
@@ -606,7 +663,21 @@ cudaError_t launch_grouped_gemms_pair(const Shape& s, const GroupedGemmArgs& a, 
     p.rows_routed = s.cap;
     p.rows_shared = s.T;
     p.wait_limit_ns = wait_limit_ns;
+    const bool split = a.down_splits > 1 && a.down_partials != nullptr && !shared &&
+                       !a.y_perm_f32;
+    if (split) {
+      p.ksplit = a.down_splits;
+      p.kit_split = (int)ceil_div(p.kit_routed, a.down_splits);
+      p.out_split = a.down_partials;
+    }
     if ((err = launch_pair<kPairDown>(m, p, num_sms, st)) != cudaSuccess) return err;
+    if (split) {
+      const int64_t n4 = (int64_t)s.cap * s.d / 4;
+      split_sum_kernel<<<(unsigned)ceil_div(n4, 256), 256, 0, st>>>(
+          a.down_partials, (int)ceil_div(p.kit_routed, p.kit_split), n4,
+          static_cast<uint16_t*>(a.y_perm));
+      if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
   }
   return cudaSuccess;
 }

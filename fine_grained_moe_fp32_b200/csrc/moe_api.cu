@@ -636,6 +636,15 @@ int dense_shape(const moe_dims* dims, Shape* s) {
 
 size_t dense_h_offset() { return al256(2 * sizeof(int32_t)); }
 
+// fp32 K-split partials of the down GEMM after h (none when it is not split)
+size_t dense_partials_offset(const Shape& s) {
+  return dense_h_offset() + region((size_t)s.T * s.I * 2);
+}
+size_t dense_partials_bytes(const Shape& s) {
+  const int sp = down_k_splits(s, kPlanSMs);
+  return sp > 1 ? region((size_t)sp * s.T * s.d * 4) : 0;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -644,7 +653,7 @@ extern "C" {
 size_t moe_dense_workspace_size(const moe_dims* dims) {
   Shape s;
   if (dense_shape(dims, &s) != MOE_OK) return 0;
-  return dense_h_offset() + region((size_t)s.T * s.I * 2);
+  return dense_partials_offset(s) + dense_partials_bytes(s);
 }
 
 int moe_dense_swiglu(const moe_dims* dims, const moe_bf16* x, const moe_bf16* w1,
@@ -677,6 +686,8 @@ int moe_dense_swiglu(const moe_dims* dims, const moe_bf16* x, const moe_bf16* w1
   a.h_perm = at<uint16_t>(workspace, dense_h_offset());
   a.y_perm = y;
   a.y_perm_f32 = false;  // the dense FFN's output is the caller's bf16 y
+  a.down_splits = down_k_splits(s, kPlanSMs);
+  if (a.down_splits > 1) a.down_partials = at<float>(workspace, dense_partials_offset(s));
   return cuda_status(
       launch_grouped_gemms(s, a, di->num_sms, di->status, g_wait_limit_ns, st, nullptr));
 }

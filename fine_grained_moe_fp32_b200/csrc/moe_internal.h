@@ -78,6 +78,10 @@ struct GroupedGemmArgs {
   // they can run while the router and the permutation do)
   enum Part : int { kAll = 0, kRoutedOnly = 1, kSharedOnly = 2 };
   int part = kAll;
+  // dense FFN at small T: the down GEMM split over K into down_splits fp32
+  // partials [down_splits, cap, d] (down_partials), summed into the bf16 y
+  int down_splits = 1;
+  float* down_partials = nullptr;
   // shared experts (S > 0 and all non-null to enable)
   const uint16_t* x;  // [T, d]
   const uint16_t *ws1, *ws3, *ws2;
@@ -100,6 +104,9 @@ bool uses_pair_gemms(const Shape& s);
 
 // ---- paired-CTA grouped GEMMs for prefill-sized segments (grouped_gemm_pair.cu)
 bool pair_gemms_supported(const Shape& s);
+// K splits of the dense FFN's down GEMM (one group, no shared experts) when
+// its tiles alone cannot fill the SM pairs; 1 otherwise
+int down_k_splits(const Shape& s, int num_sms);
 cudaError_t launch_grouped_gemms_pair(const Shape& s, const GroupedGemmArgs& a, int num_sms,
                                       unsigned int* status, uint64_t wait_limit_ns,
                                       cudaStream_t st, cudaEvent_t between);

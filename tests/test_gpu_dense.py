@@ -34,6 +34,9 @@ CASES = [
     ("T37_pairs_ragged", 37, 256, 256),
     ("T300_pairs", 300, 512, 384),
     ("T200_one_cta_I192", 200, 256, 192),
+    # too few down tiles for the SM pairs: the down GEMM is split over K
+    ("T128_down_split_4", 128, 512, 1024),
+    ("T300_down_split_ragged", 300, 512, 1408),
 ]
 
 
@@ -54,6 +57,16 @@ def test_dense_full_size_sampled():
     idx = torch.as_tensor(toks, device="cuda")
     ref = O.dense_swiglu(inp["x"][idx].cpu(), inp["w1"].cpu(), inp["w3"].cpu(), inp["w2"].cpu())
     PU.check_output(y[idx], ref, "dense y (sampled)", spec=False)
+
+
+def test_dense_full_size_T128_down_split():
+    """d = 5120, I = 11264 at T = 128: the down GEMM's 20 tiles are split
+    over K (fp32 partials summed in a fixed order, one rounding); every
+    token against the oracle."""
+    inp = make_dense_inputs(128, 5120, DENSE_I, device="cuda")
+    y = _run(inp)
+    ref = O.dense_swiglu(inp["x"].cpu(), inp["w1"].cpu(), inp["w3"].cpu(), inp["w2"].cpu())
+    PU.check_output(y, ref, "dense y (T=128)", spec=False)
 
 
 def test_dense_empty_batch():
