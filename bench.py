@@ -192,14 +192,28 @@ def train_gemm_flops(cfg, T):
             "wgrad_w2": down, "dgrad_up": up, "wgrad_w1_w3": up}
 
 
-def gemm_units(cfg, T, counts):
+def shared_on_side_stream(cfg, T, train):
+    """The inference forward of prefill-sized batches runs the shared experts'
+    GEMMs on the library's side stream (beside the permutation), so the
+    gate/up and down phases timed on the caller's stream hold the routed
+    experts' GEMMs only (the paired-CTA kernels: T*k > 24*E)."""
+    return (not train) and cfg.S > 0 and T * cfg.k > 24 * cfg.E and cfg.I % 128 == 0 \
+        and cfg.d % 256 == 0
+
+
+def gemm_units(cfg, T, counts, routed_only=False):
     """Algorithmic work of the two grouped GEMMs for one step (padding not
-    counted): bytes that must move and flops that must be done."""
+    counted): bytes that must move and flops that must be done; with
+    ``routed_only`` the routed experts' launches alone."""
     d, I, S, k = cfg.d, cfg.I, cfg.S, cfg.k
     touched = int((counts > 0).sum())
     rows = T * k
-    g1_bytes = (touched + S) * 2 * I * d * 2 + (rows + T) * d * 2 + (rows + T * S) * I * 2
-    g2_bytes = (touched + S) * d * I * 2 + (rows + T * S) * I * 2 + rows * d * 4 + T * d * 4
+    if routed_only:
+        S = 0
+    g1_bytes = (touched + S) * 2 * I * d * 2 + (rows + (T if S else 0)) * d * 2 \
+        + (rows + T * S) * I * 2
+    g2_bytes = (touched + S) * d * I * 2 + (rows + T * S) * I * 2 + rows * d * 4 \
+        + (T * d * 4 if S else 0)
     g1_flops = 2 * (rows * 2 * I + T * 2 * S * I) * d
     g2_flops = 2 * (rows * I + T * S * I) * d
     return {"touched_experts": touched, "gemm_gate_up_swiglu": (g1_bytes, g1_flops),
@@ -402,7 +416,8 @@ def measure(cfg, args, dev, world, rank, local):
     if train:
         phase_ms["balance_stats_bias_step"] = statistics.mean(
             bal_ev[s][0].elapsed_time(bal_ev[s][1]) for s in range(n_phase))
-    units = gemm_units(cfg, T, counts)
+    split = shared_on_side_stream(cfg, T, train)
+    units = gemm_units(cfg, T, counts, routed_only=split)
     if train:
         tflops = train_gemm_flops(cfg, T)
         dom = max(tflops, key=lambda n: phase_ms[n])
@@ -520,7 +535,8 @@ def measure(cfg, args, dev, world, rank, local):
         peak = peaks["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak}
-    roof["kernel"] = dom
+    roof["kernel"] = dom + (" (routed experts; the shared experts' GEMMs run on a side stream)"
+                            if split else "")
     roof["kernel_ms"] = dom_ms
     roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if hbm_bound else 'bf16_tflops'})"
     roof["traffic"] = load_traffic(dom, cfg.name)
@@ -543,7 +559,7 @@ def measure(cfg, args, dev, world, rank, local):
                    "d2h_bytes_per_step": T * cfg.d * 2},
            "gpu_launches": (forward_kernels(T) + (BWD_KERNELS + BALANCE_KERNELS if train else 0))
            * args.steps,
-           "config": config_dict(cfg, world, args.align, units["touched_experts"]),
+           "config": config_dict(cfg, world, args.align, gemm_units(cfg, T, counts)["touched_experts"]),
            "n_phase": n_phase}
     if train:
         res["train_tflop_per_step"] = sum(train_gemm_flops(cfg, T).values()) / 1e12
