@@ -392,38 +392,46 @@ int forward_impl(const moe_dims* dims, const moe_bf16* x, const float* w_gate, c
     a.g_shared = at<float>(ws, TL.g_shared);
     a.u_shared = at<float>(ws, TL.u_shared);
   }
-  // Prefill-sized batches: the shared experts' GEMMs do not depend on the
-  // routing.  After the router they go to the side stream, launched before
-  // the permutation so their CTAs are resident first: the permutation's
-  // HBM-bound gather then runs on the SMs beside those compute-bound GEMMs.
-  // The caller's stream waits for them before the combine.  Measured on the
-  // same box against one stream: 2.6 % faster at T = 4096, 1.3 % at 16384;
-  // the training forward (which also stores g and u) was 1.2 % slower, so
-  // it keeps one stream.
-  const bool split = !train && s.S > 0 && s.T > 0 && uses_pair_gemms(s);
+  // The shared experts' GEMMs do not depend on the routing, so the inference
+  // forward runs them on the library's side stream and the caller's stream
+  // waits for them (one event) before the combine.
+  //  * Prefill-sized batches: launched after the router, before the
+  //    permutation, on every SM: their CTAs are resident first and the
+  //    permutation's HBM-bound row copy runs beside those compute-bound
+  //    GEMMs.  Same-box A/B against one stream: 2.6 % faster at T = 4096,
+  //    1.3 % at 16384; the training forward (which also stores g and u) was
+  //    1.2 % slower, so it keeps one stream.
+  //  * Decode-sized batches: launched before the router on half of the SMs,
+  //    so the shared weights stream while the latency-bound router and
+  //    permutation run on the other half.
+  const bool pair = uses_pair_gemms(s);
+  const bool split = !train && s.S > 0 && s.T > 0;
   std::unique_lock<std::mutex> fork_lock(g_fork_mu, std::defer_lock);
   NvtxRange call(train ? "moe_forward_train" : "moe_forward");
   NvtxPhases ph;
-  ph.next("router");
-  cudaError_t e = phase(0, st);
-  if (e == cudaSuccess)
-    e = launch_router(s, x, w_gate, bias, probs, idx, wts, at<float>(ws, L.route_partials),
-                      kPlanSMs, st);
-  if (e == cudaSuccess) e = phase(1, st);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
-  if (split) {
+  cudaError_t e = cudaSuccess;
+  auto fork_shared = [&](int ctas) {
     ph.next("shared_experts (side stream)");
     fork_lock.lock();
     GroupedGemmArgs sh = a;
     sh.part = GroupedGemmArgs::kSharedOnly;
     if ((e = cudaEventRecord(di->fork, st)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(di->side, di->fork, 0)) != cudaSuccess ||
-        (e = launch_grouped_gemms(s, sh, di->num_sms, di->status, g_wait_limit_ns, di->side)) !=
+        (e = launch_grouped_gemms(s, sh, ctas, di->status, g_wait_limit_ns, di->side)) !=
             cudaSuccess ||
         (e = cudaEventRecord(di->join, di->side)) != cudaSuccess)
-      return MOE_ERR_CUDA;
+      return false;
     a.part = GroupedGemmArgs::kRoutedOnly;
-  }
+    return true;
+  };
+  if ((e = phase(0, st)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (split && !pair && !fork_shared(di->num_sms / 2)) return MOE_ERR_CUDA;
+  ph.next("router");
+  e = launch_router(s, x, w_gate, bias, probs, idx, wts, at<float>(ws, L.route_partials),
+                    kPlanSMs, st);
+  if (e == cudaSuccess) e = phase(1, st);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (split && pair && !fork_shared(di->num_sms)) return MOE_ERR_CUDA;
   ph.next("permute");
   e = launch_permute(s, idx, x, counts, offsets, row_of, tor, x_perm,
                      at<void>(ws, L.permute_scratch), di->status, st);

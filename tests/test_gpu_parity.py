@@ -368,12 +368,13 @@ def test_forward_full_size_every_segment(cfg):
 
 
 @pytest.mark.parametrize("cfg,T", [(small_config(T=700, d=512, E=16, k=4, I=256), None),
-                                   (PREFILL_BALANCED, None)],
-                         ids=["pair_prefill_T700", "prefill_balanced"])
-def test_fused_prefill_forward_equals_the_step_calls(cfg, T):
-    """At prefill sizes moe_forward runs the shared experts' GEMMs on a side
-    stream beside the permutation and launches the routed GEMMs alone; the
-    result must be bit-identical to the public step calls (moe_route,
+                                   (PREFILL_BALANCED, None), (DECODE, None), (TINY, None)],
+                         ids=["pair_prefill_T700", "prefill_balanced", "decode", "tiny"])
+def test_fused_forward_equals_the_step_calls(cfg, T):
+    """moe_forward runs the shared experts' GEMMs on a side stream (beside
+    the permutation at prefill sizes, beside the router and the permutation
+    on half of the SMs at decode sizes) and launches the routed GEMMs alone;
+    the result must be bit-identical to the public step calls (moe_route,
     moe_permute, moe_grouped_swiglu, moe_combine) on the same batch, whose
     grouped-GEMM call runs the routed experts in one launch per projection.
     The combine is fed the fused call's fp32 shared output."""
