@@ -65,8 +65,11 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+# the kernel, its PTX helpers, and the entry point that decides what one
+# launch covers (a change to any of them invalidates a traffic capture)
 GEMM_SOURCES = ("fine_grained_moe_fp32_b200/csrc/grouped_gemm.cu",
-                "fine_grained_moe_fp32_b200/csrc/ptx_sm100.cuh")
+                "fine_grained_moe_fp32_b200/csrc/ptx_sm100.cuh",
+                "fine_grained_moe_fp32_b200/csrc/moe_api.cu")
 
 
 def kernel_source_hash() -> str:
@@ -193,12 +196,11 @@ def train_gemm_flops(cfg, T):
 
 
 def shared_on_side_stream(cfg, T, train):
-    """The inference forward of prefill-sized batches runs the shared experts'
-    GEMMs on the library's side stream (beside the permutation), so the
-    gate/up and down phases timed on the caller's stream hold the routed
-    experts' GEMMs only (the paired-CTA kernels: T*k > 24*E)."""
-    return (not train) and cfg.S > 0 and T * cfg.k > 24 * cfg.E and cfg.I % 128 == 0 \
-        and cfg.d % 256 == 0
+    """The inference forward runs the shared experts' GEMMs on the library's
+    side stream (beside the router and the permutation), so the gate/up and
+    down phases timed on the caller's stream hold the routed experts' GEMMs
+    only."""
+    return (not train) and cfg.S > 0 and T > 0
 
 
 def gemm_units(cfg, T, counts, routed_only=False):
