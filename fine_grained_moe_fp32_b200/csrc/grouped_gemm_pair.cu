@@ -12,10 +12,7 @@
 //    which reads A and B from both CTAs' shared memory and leaves each CTA's
 //    128 output rows in its own TMEM.  Per SM this halves the token bytes
 //    loaded per flop.  The weights (from HBM) and the token rows (from L2)
-//    have separate smem rings and producers (6 and 7 stages of 16 KB): the
-//    token rows are re-read from L2 by every feature tile of a segment and
-//    their latency, not the HBM weight stream, is what stalls the MMA when
-//    the two share one shallow ring (measured with per-role wait counters).
+//    have separate producer warps that fill one ring of three 64 KB stages.
 //  * Both CTAs' TMA loads complete on the leader's "full" barrier (the
 //    leader arms it with the pair's byte count); the leader's MMA commits
 //    arrive on the "empty" / "tmem full" barriers of both CTAs at once; both
