@@ -25,59 +25,80 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 constexpr int kCbThreads = 128;
-constexpr int kMaxVecPerThread = 8;  // d <= 8 * 8 * 128 = 8192
 
-// One CTA per token.  The dot products are reduced in a fixed order (per
-// thread, then warp butterfly, then warps in order), so dw is deterministic.
+// One CTA per token.  Each thread takes its 16-byte vectors of dy[t] in turn
+// and, for each, issues the loads of all k routed rows before using them (the
+// k rows are independent streams, so their HBM latencies overlap).  The dot
+// products are reduced in a fixed order (per thread over its vectors, then
+// warp butterfly, then warps in order), so dw is deterministic.
+constexpr int kCbMaxK = 8;
+
 __global__ void __launch_bounds__(kCbThreads)
 combine_bwd_kernel(const uint16_t* __restrict__ dy, const float* __restrict__ y_perm,
                    const int32_t* __restrict__ row_of, const float* __restrict__ topk_w,
                    uint16_t* __restrict__ dy_perm, float* __restrict__ dw, int d, int k,
                    int64_t cap) {
   const int t = blockIdx.x;
-  __shared__ float red[kCbThreads / 32];
-  const int nv = d / 8;
-  uint4 g[kMaxVecPerThread];
-#pragma unroll
-  for (int i = 0; i < kMaxVecPerThread; ++i) {
-    const int v = threadIdx.x + i * kCbThreads;
-    g[i] = v < nv ? reinterpret_cast<const uint4*>(dy + (size_t)t * d)[v] : make_uint4(0, 0, 0, 0);
-  }
-  for (int j = 0; j < k; ++j) {
+  __shared__ float red[kCbMaxK][kCbThreads / 32];
+  __shared__ const float* yrow[kCbMaxK];
+  __shared__ uint16_t* orow[kCbMaxK];
+  __shared__ float wsel[kCbMaxK];
+  if ((int)threadIdx.x < k) {
+    const int j = threadIdx.x;
     const int r = row_of[(size_t)t * k + j];
-    const float w = topk_w[(size_t)t * k + j];
-    float part = 0.f;
-    if (MOE_CHECK(r >= -1 && r < cap) && r >= 0 && r < cap) {
-      const float4* yr = reinterpret_cast<const float4*>(y_perm + (size_t)r * d);
-      uint4* out = reinterpret_cast<uint4*>(dy_perm + (size_t)r * d);
+    const bool ok = MOE_CHECK(r >= -1 && r < cap) && r >= 0 && r < cap;  // -1: pair skipped
+    yrow[j] = ok ? y_perm + (size_t)r * d : nullptr;
+    orow[j] = ok ? dy_perm + (size_t)r * d : nullptr;
+    wsel[j] = topk_w[(size_t)t * k + j];
+  }
+  __syncthreads();
+  const int nv = d / 8;
+  float part[kCbMaxK];
 #pragma unroll
-      for (int i = 0; i < kMaxVecPerThread; ++i) {
-        const int v = threadIdx.x + i * kCbThreads;
-        if (v < nv) {
-          const float4 ya = yr[2 * v], yb = yr[2 * v + 1];
-          const uint32_t gw[4] = {g[i].x, g[i].y, g[i].z, g[i].w};
-          const float yv[8] = {ya.x, ya.y, ya.z, ya.w, yb.x, yb.y, yb.z, yb.w};
-          uint32_t o[4];
+  for (int j = 0; j < kCbMaxK; ++j) part[j] = 0.f;
+#pragma unroll 1
+  for (int v = threadIdx.x; v < nv; v += kCbThreads) {
+    const uint4 gv = reinterpret_cast<const uint4*>(dy + (size_t)t * d)[v];
+    float4 ya[kCbMaxK], yb[kCbMaxK];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            part = fmaf(bf16lo(gw[q]), yv[2 * q], part);
-            part = fmaf(bf16hi(gw[q]), yv[2 * q + 1], part);
-            o[q] = pack_bf16(w * bf16lo(gw[q]), w * bf16hi(gw[q]));
-          }
-          out[v] = make_uint4(o[0], o[1], o[2], o[3]);
-        }
+    for (int j = 0; j < kCbMaxK; ++j) {
+      if (j < k && yrow[j] != nullptr) {
+        const float4* yr = reinterpret_cast<const float4*>(yrow[j]);
+        ya[j] = __ldg(yr + 2 * v);
+        yb[j] = __ldg(yr + 2 * v + 1);
       }
     }
+    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = part;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float s = 0.f;
-      for (int i = 0; i < kCbThreads / 32; ++i) s += red[i];
-      dw[(size_t)t * k + j] = s;
+    for (int j = 0; j < kCbMaxK; ++j) {
+      if (j < k && yrow[j] != nullptr) {
+        const float yv[8] = {ya[j].x, ya[j].y, ya[j].z, ya[j].w,
+                             yb[j].x, yb[j].y, yb[j].z, yb[j].w};
+        const float w = wsel[j];
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          part[j] = fmaf(bf16lo(gw[q]), yv[2 * q], part[j]);
+          part[j] = fmaf(bf16hi(gw[q]), yv[2 * q + 1], part[j]);
+          o[q] = pack_bf16(w * bf16lo(gw[q]), w * bf16hi(gw[q]));
+        }
+        reinterpret_cast<uint4*>(orow[j])[v] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
     }
-    __syncthreads();
+  }
+#pragma unroll
+  for (int j = 0; j < kCbMaxK; ++j) {
+    if (j < k) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) part[j] += __shfl_xor_sync(0xffffffffu, part[j], o);
+      if ((threadIdx.x & 31) == 0) red[j][threadIdx.x >> 5] = part[j];
+    }
+  }
+  __syncthreads();
+  if ((int)threadIdx.x < k) {
+    float s = 0.f;
+    for (int i = 0; i < kCbThreads / 32; ++i) s += red[threadIdx.x][i];
+    dw[(size_t)t * k + threadIdx.x] = s;
   }
 }
 
