@@ -144,6 +144,8 @@ CASES = [
     # ~512 rows per expert: weight gradients with the A panel resident (<= 512
     # rows) and with 512-row panels reloaded per N tile (longer segments)
     ("E4_k1_T2048_panels_over_512", small_config(T=2048, d=256, E=4, k=1, I=128), None),
+    # hidden size past 8192: every 16-byte vector of a token's row, not a fixed count per thread
+    ("E8_k2_T64_d8448_wide_rows", small_config(T=64, d=8448, E=8, k=2, I=128), None),
 ]
 
 
