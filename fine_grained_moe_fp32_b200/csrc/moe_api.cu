@@ -401,9 +401,12 @@ int forward_impl(const moe_dims* dims, const moe_bf16* x, const float* w_gate, c
   //    GEMMs.  Same-box A/B against one stream: 2.6 % faster at T = 4096,
   //    1.3 % at 16384; the training forward (which also stores g and u) was
   //    1.2 % slower, so it keeps one stream.
-  //  * Decode-sized batches: launched before the router on half of the SMs,
-  //    so the shared weights stream while the latency-bound router and
-  //    permutation run on the other half.
+  //  * Decode-sized batches: launched before the router on two thirds of the
+  //    SMs, so the shared weights stream while the latency-bound router and
+  //    permutation run on the rest.  With T = 128 the shared gate/up GEMM has
+  //    88 tiles: on half of the SMs it took two waves and held SMs into the
+  //    routed gate/up GEMM (same-box A/B, per step: 74 CTAs 0.923-0.930 ms,
+  //    100 CTAs 0.915-0.919, 112 CTAs 0.919-0.921, 148 CTAs 0.921-0.923).
   const bool pair = uses_pair_gemms(s);
   const bool split = !train && s.S > 0 && s.T > 0;
   std::unique_lock<std::mutex> fork_lock(g_fork_mu, std::defer_lock);
@@ -425,7 +428,7 @@ int forward_impl(const moe_dims* dims, const moe_bf16* x, const float* w_gate, c
     return true;
   };
   if ((e = phase(0, st)) != cudaSuccess) return MOE_ERR_CUDA;
-  if (split && !pair && !fork_shared(di->num_sms / 2)) return MOE_ERR_CUDA;
+  if (split && !pair && !fork_shared(di->num_sms * 2 / 3)) return MOE_ERR_CUDA;
   ph.next("router");
   e = launch_router(s, x, w_gate, bias, probs, idx, wts, at<float>(ws, L.route_partials),
                     kPlanSMs, st);
