@@ -411,6 +411,15 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
                 out[(size_t)(t.row0 + c0 + j) * p.ld_shared + col] =
                     __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
           }
+        } else if (routed && p.ksplit > 1) {
+          // one K split's fp32 pre-activations: g from the gate lanes (q < 2),
+          // u from the up lanes, as planes 0 and 1 of the split's partial
+          const int col = t.ft * 128 + (int)rank * 64 + (frow & 63);
+          float* out = p.out_split +
+                       ((size_t)t.ks * 2 + (q < 2 ? 0 : 1)) * p.rows_routed * p.ld_routed;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < nj) out[(size_t)(t.row0 + c0 + j) * p.ld_routed + col] = __uint_as_float(v[j]);
         } else {
           // the gate lanes (q < 2) stage g, the up lanes (q >= 2) stage u;
           // then each pair of warps finishes half of the chunk's tokens for
@@ -559,25 +568,56 @@ __global__ void split_sum_kernel(const float* __restrict__ part, int splits, int
                                               *reinterpret_cast<const uint32_t*>(&hi));
 }
 
-}  // namespace
+// h[i] = bf16(silu(g) * u) with g and u the fp32 sums over the K splits of
+// part[s][0][i] and part[s][1][i], s ascending (plane = n4 float4s).
+__global__ void split_swiglu_kernel(const float* __restrict__ part, int splits, int64_t n4,
+                                    uint16_t* __restrict__ h) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  const float4* p4 = reinterpret_cast<const float4*>(part);
+  float4 g = p4[i], u = p4[n4 + i];
+  for (int sp = 1; sp < splits; ++sp) {
+    const float4 a = p4[(size_t)sp * 2 * n4 + i], b = p4[(size_t)sp * 2 * n4 + n4 + i];
+    g.x += a.x; g.y += a.y; g.z += a.z; g.w += a.w;
+    u.x += b.x; u.y += b.y; u.z += b.z; u.w += b.w;
+  }
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(psilu(g.x) * u.x, psilu(g.y) * u.y);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(psilu(g.z) * u.z, psilu(g.w) * u.w);
+  reinterpret_cast<uint2*>(h)[i] = make_uint2(*reinterpret_cast<const uint32_t*>(&lo),
+                                              *reinterpret_cast<const uint32_t*>(&hi));
+}
 
-int down_k_splits(const Shape& s, int num_sms) {
-  if (!uses_pair_gemms(s) || s.S > 0 || s.E != 1) return 1;
+// K splits for a GEMM of `base` pair tiles of `kit` K chunks each: the fewest
+// splits among those with the least (waves x K chunks per tile).  Only a GEMM
+// of at most two waves of pair tiles is split, and only when that cuts the
+// cost by 15 % or more: the fp32 partials take a round trip through HBM.
+int plan_k_splits(int base, int kit, int num_sms) {
   const int pairs = num_sms / 2;
-  const int base = (int)ceil_div(s.T, kNT) * (s.d / 256);
-  const int kit = s.I / kBK;
-  if (base >= pairs || kit < 4) return 1;
-  // fewest splits among those with the least (waves x K chunks per tile)
+  if (pairs <= 0 || base > 2 * pairs || kit < 4) return 1;
   int best = 1;
-  int64_t best_cost = ceil_div(base, pairs) * kit;
+  const int64_t unsplit = ceil_div(base, pairs) * kit;
+  int64_t best_cost = unsplit;
   for (int sp = 2; sp <= 8 && sp <= kit / 2; ++sp) {
+    if (ceil_div(kit, sp) * (sp - 1) >= kit) continue;  // every split gets K chunks
     const int64_t cost = ceil_div((int64_t)base * sp, pairs) * ceil_div(kit, sp);
     if (cost < best_cost) {
       best_cost = cost;
       best = sp;
     }
   }
-  return best;
+  return best_cost * 100 <= unsplit * 85 ? best : 1;
+}
+
+}  // namespace
+
+int down_k_splits(const Shape& s, int num_sms) {
+  if (!uses_pair_gemms(s) || s.S > 0 || s.E != 1) return 1;
+  return plan_k_splits((int)ceil_div(s.T, kNT) * (s.d / 256), s.I / kBK, num_sms);
+}
+
+int up_k_splits(const Shape& s, int num_sms) {
+  if (!uses_pair_gemms(s) || s.S > 0 || s.E != 1) return 1;
+  return plan_k_splits((int)ceil_div(s.T, kNT) * (s.I / 128), s.d / kBK, num_sms);
 }
 
 cudaError_t launch_grouped_gemms_pair(const Shape& s, const GroupedGemmArgs& a, int num_sms,
@@ -625,7 +665,20 @@ cudaError_t launch_grouped_gemms_pair(const Shape& s, const GroupedGemmArgs& a, 
     p.rows_routed = s.cap;
     p.rows_shared = s.T;
     p.wait_limit_ns = wait_limit_ns;
+    const bool split = a.up_splits > 1 && a.up_partials != nullptr && !shared &&
+                       a.g_perm == nullptr;
+    if (split) {
+      p.ksplit = a.up_splits;
+      p.kit_split = (int)ceil_div(p.kit_routed, a.up_splits);
+      p.out_split = a.up_partials;
+    }
     if ((err = launch_pair<kPairSwiGLU>(m, p, num_sms, st)) != cudaSuccess) return err;
+    if (split) {
+      const int64_t n4 = (int64_t)s.cap * s.I / 4;
+      split_swiglu_kernel<<<(unsigned)ceil_div(n4, 256), 256, 0, st>>>(
+          a.up_partials, (int)ceil_div(p.kit_routed, p.kit_split), n4, a.h_perm);
+      if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
     if (between != nullptr && (err = cudaEventRecord(between, st)) != cudaSuccess) return err;
   }
   // ---- down GEMM: a pair tile = 256 output features x up to 256 tokens

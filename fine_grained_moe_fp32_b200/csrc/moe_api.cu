@@ -651,9 +651,12 @@ size_t dense_h_offset() { return al256(2 * sizeof(int32_t)); }
 size_t dense_partials_offset(const Shape& s) {
   return dense_h_offset() + region((size_t)s.T * s.I * 2);
 }
+// (the gate/up GEMM's K-split partials use the same memory first)
 size_t dense_partials_bytes(const Shape& s) {
-  const int sp = down_k_splits(s, kPlanSMs);
-  return sp > 1 ? region((size_t)sp * s.T * s.d * 4) : 0;
+  const int sd = down_k_splits(s, kPlanSMs), su = up_k_splits(s, kPlanSMs);
+  const size_t down = sd > 1 ? (size_t)sd * s.T * s.d * 4 : 0;
+  const size_t up = su > 1 ? (size_t)su * 2 * s.T * s.I * 4 : 0;
+  return down > 0 || up > 0 ? region(std::max(down, up)) : 0;
 }
 
 }  // namespace
@@ -699,6 +702,8 @@ int moe_dense_swiglu(const moe_dims* dims, const moe_bf16* x, const moe_bf16* w1
   a.y_perm_f32 = false;  // the dense FFN's output is the caller's bf16 y
   a.down_splits = down_k_splits(s, kPlanSMs);
   if (a.down_splits > 1) a.down_partials = at<float>(workspace, dense_partials_offset(s));
+  a.up_splits = up_k_splits(s, kPlanSMs);
+  if (a.up_splits > 1) a.up_partials = at<float>(workspace, dense_partials_offset(s));
   return cuda_status(
       launch_grouped_gemms(s, a, di->num_sms, di->status, g_wait_limit_ns, st, nullptr));
 }

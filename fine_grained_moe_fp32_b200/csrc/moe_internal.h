@@ -82,6 +82,11 @@ struct GroupedGemmArgs {
   // partials [down_splits, cap, d] (down_partials), summed into the bf16 y
   int down_splits = 1;
   float* down_partials = nullptr;
+  // dense FFN at small T: the gate/up GEMM split over K into up_splits fp32
+  // partials [up_splits, 2 (g, u), cap, I] (up_partials), summed in order
+  // before the SwiGLU (it is not linear); may share down_partials' memory
+  int up_splits = 1;
+  float* up_partials = nullptr;
   // shared experts (S > 0 and all non-null to enable)
   const uint16_t* x;  // [T, d]
   const uint16_t *ws1, *ws3, *ws2;
@@ -107,6 +112,7 @@ bool pair_gemms_supported(const Shape& s);
 // K splits of the dense FFN's down GEMM (one group, no shared experts) when
 // its tiles alone cannot fill the SM pairs; 1 otherwise
 int down_k_splits(const Shape& s, int num_sms);
+int up_k_splits(const Shape& s, int num_sms);
 cudaError_t launch_grouped_gemms_pair(const Shape& s, const GroupedGemmArgs& a, int num_sms,
                                       unsigned int* status, uint64_t wait_limit_ns,
                                       cudaStream_t st, cudaEvent_t between);

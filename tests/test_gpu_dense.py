@@ -34,7 +34,9 @@ CASES = [
     ("T37_pairs_ragged", 37, 256, 256),
     ("T300_pairs", 300, 512, 384),
     ("T200_one_cta_I192", 200, 256, 192),
-    # too few down tiles for the SM pairs: the down GEMM is split over K
+    # too few tiles for the SM pairs: the gate/up GEMM (2 K splits: fp32 g and
+    # u partials summed before the SwiGLU) and the down GEMM are split over K
+    # (T300_pairs: the gate/up GEMM alone)
     ("T128_down_split_4", 128, 512, 1024),
     ("T300_down_split_ragged", 300, 512, 1408),
 ]
@@ -60,9 +62,10 @@ def test_dense_full_size_sampled():
 
 
 def test_dense_full_size_T128_down_split():
-    """d = 5120, I = 11264 at T = 128: the down GEMM's 20 tiles are split
-    over K (fp32 partials summed in a fixed order, one rounding); every
-    token against the oracle."""
+    """d = 5120, I = 11264 at T = 128: the gate/up GEMM's 88 tiles (5 K
+    splits) and the down GEMM's 20 tiles (7 K splits) are split over K (fp32
+    partials summed in a fixed order, one rounding each); every token
+    against the oracle."""
     inp = make_dense_inputs(128, 5120, DENSE_I, device="cuda")
     y = _run(inp)
     ref = O.dense_swiglu(inp["x"].cpu(), inp["w1"].cpu(), inp["w3"].cpu(), inp["w2"].cpu())
