@@ -413,39 +413,50 @@ int forward_impl(const moe_dims* dims, const moe_bf16* x, const float* w_gate, c
   NvtxRange call(train ? "moe_forward_train" : "moe_forward");
   NvtxPhases ph;
   cudaError_t e = cudaSuccess;
+  bool forked = false;
   auto fork_shared = [&](int ctas) {
     ph.next("shared_experts (side stream)");
     fork_lock.lock();
     GroupedGemmArgs sh = a;
     sh.part = GroupedGemmArgs::kSharedOnly;
     if ((e = cudaEventRecord(di->fork, st)) != cudaSuccess ||
-        (e = cudaStreamWaitEvent(di->side, di->fork, 0)) != cudaSuccess ||
-        (e = launch_grouped_gemms(s, sh, ctas, di->status, g_wait_limit_ns, di->side)) !=
-            cudaSuccess ||
-        (e = cudaEventRecord(di->join, di->side)) != cudaSuccess)
+        (e = cudaStreamWaitEvent(di->side, di->fork, 0)) != cudaSuccess)
       return false;
+    forked = true;
+    e = launch_grouped_gemms(s, sh, ctas, di->status, g_wait_limit_ns, di->side);
+    // recorded whatever the launch did, so the caller's stream can always be
+    // ordered after the side stream's work
+    const cudaError_t ej = cudaEventRecord(di->join, di->side);
+    if (e == cudaSuccess) e = ej;
+    if (e != cudaSuccess) return false;
     a.part = GroupedGemmArgs::kRoutedOnly;
     return true;
   };
+  // an error after the fork still orders the caller's stream after the side
+  // stream's kernels, which write the caller's workspace
+  auto fail = [&]() {
+    if (forked) cudaStreamWaitEvent(st, di->join, 0);
+    return MOE_ERR_CUDA;
+  };
   if ((e = phase(0, st)) != cudaSuccess) return MOE_ERR_CUDA;
-  if (split && !pair && !fork_shared(di->num_sms * 2 / 3)) return MOE_ERR_CUDA;
+  if (split && !pair && !fork_shared(di->num_sms * 2 / 3)) return fail();
   ph.next("router");
   e = launch_router(s, x, w_gate, bias, probs, idx, wts, at<float>(ws, L.route_partials),
                     kPlanSMs, st);
   if (e == cudaSuccess) e = phase(1, st);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
-  if (split && pair && !fork_shared(di->num_sms)) return MOE_ERR_CUDA;
+  if (e != cudaSuccess) return fail();
+  if (split && pair && !fork_shared(di->num_sms)) return fail();
   ph.next("permute");
   e = launch_permute(s, idx, x, counts, offsets, row_of, tor, x_perm,
                      at<void>(ws, L.permute_scratch), di->status, st);
   if (e == cudaSuccess) e = phase(2, st);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (e != cudaSuccess) return fail();
   ph.next("grouped_gemms");
   e = launch_grouped_gemms(s, a, di->num_sms, di->status, g_wait_limit_ns, st,
                            g_phase_on ? g_phase_events[3] : nullptr);
   if (e == cudaSuccess) e = phase(4, st);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
-  if (split && (e = cudaStreamWaitEvent(st, di->join, 0)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (e != cudaSuccess) return fail();
+  if (forked && (e = cudaStreamWaitEvent(st, di->join, 0)) != cudaSuccess) return MOE_ERR_CUDA;
   ph.next("combine");
   e = launch_combine(s, y_perm, row_of, wts, s.S > 0 ? y_sh : nullptr, y, st);
   if (e == cudaSuccess) e = phase(5, st);
