@@ -40,8 +40,8 @@ struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
   unsigned int* status = nullptr;
-  // prefill forward: the shared experts' GEMMs run on `side` while the
-  // router and the permutation run on the caller's stream (fork, join)
+  // inference forward: the shared experts' GEMMs run on `side` beside the
+  // router and the permutation on the caller's stream (fork, join)
   cudaStream_t side = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
 };
@@ -84,8 +84,15 @@ const DeviceInfo* device_info() {
     if (checks_init_all(d.status) != cudaSuccess) return nullptr;
     if (cudaStreamCreateWithFlags(&d.side, cudaStreamNonBlocking) != cudaSuccess ||
         cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&d.join, cudaEventDisableTiming) != cudaSuccess)
+        cudaEventCreateWithFlags(&d.join, cudaEventDisableTiming) != cudaSuccess) {
+      // leave nothing half made: the next call starts over
+      if (d.join != nullptr) cudaEventDestroy(d.join);
+      if (d.fork != nullptr) cudaEventDestroy(d.fork);
+      if (d.side != nullptr) cudaStreamDestroy(d.side);
+      d.side = nullptr;
+      d.fork = d.join = nullptr;
       return nullptr;
+    }
     d.ready = true;
   }
   return &d;
