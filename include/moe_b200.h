@@ -313,7 +313,10 @@ int moe_backward_f32(const moe_dims* dims, const moe_bf16* x, const float* w_gat
  *              n_shared and align are ignored.  d % 128 == 0, I % 64 == 0.
  *   x  [T, d]  bf16;  w1, w3 [I, d], w2 [d, I] bf16
  *   y  [T, d]  bf16 out (h rounded to bf16, fp32 accumulation, one rounding)
- *   workspace  moe_dense_workspace_size() bytes, 256-byte aligned (h [T, I]).
+ *   workspace  moe_dense_workspace_size() bytes, 256-byte aligned: h [T, I],
+ *              and at small T (too few tiles for the SMs) the fp32 partial
+ *              sums of a GEMM split over K, added in a fixed order before the
+ *              SwiGLU (gate/up) or the one rounding of y (down).
  * Returns INVALID_ARG (null or misaligned pointer), UNSUPPORTED_SHAPE,
  * WORKSPACE, CUDA.  T == 0 is a no-op.
  * ---------------------------------------------------------------------- */
