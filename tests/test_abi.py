@@ -132,6 +132,22 @@ def test_dense_calls_rejected_on_host(lib):
                                 None) == M.MOE_ERR_WORKSPACE
 
 
+def test_dense_workspace_holds_the_split_k_partials(lib):
+    """At T = 128 (d = 5120, I = 11264) both dense GEMMs have too few pair
+    tiles for 74 SM pairs and are split over K: 5 splits of fp32 g and u
+    partials for gate/up, 7 of fp32 y partials for down, sharing one region
+    after h.  The workspace must hold h and the larger of the two; at T =
+    4096 nothing is split and the workspace is h alone (plus alignment)."""
+    def need(T):
+        return lib.moe_dense_workspace_size(ctypes.byref(M.dense_dims(T=T, d=5120, I=11264)))
+    T, d, I = 128, 5120, 11264
+    h = T * I * 2
+    up, down = 5 * 2 * T * I * 4, 7 * T * d * 4
+    assert need(T) >= h + max(up, down)
+    assert need(T) < h + max(up, down) + 4096
+    assert 4096 * I * 2 <= need(4096) < 4096 * I * 2 + 4096
+
+
 def test_expert_parallel_sizes_and_rejects_on_host(lib):
     fake = ctypes.c_void_p(1 << 20)   # never dereferenced: every call below fails first
     dm = M.dims(T=128, d=5120, E=128, k=6, I=1408, n_shared=2, align=16)
