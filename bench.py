@@ -38,11 +38,37 @@ from fine_grained_moe_fp32_b200.workloads import CONFIGS, make_inputs  # noqa: E
 
 METRIC = "MoE-layer tokens/s (bf16, d=5120, 128E top-6 + 2 shared) and % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-def forward_kernels(T: int) -> int:
+def forward_kernels(T: int, side: bool = False) -> int:
     """Launches of one moe_forward: router GEMM + top-k, the permutation (one
     index kernel + row copy for a batch of at most 256 tokens, else count,
-    scan, scatter + row copy), the two grouped GEMMs, the combine."""
-    return 2 + (2 if T <= 256 else 4) + 2 + 1
+    scan, scatter + row copy), the two grouped GEMMs, the combine; with
+    ``side`` the shared experts' two GEMMs launched on the side stream."""
+    return 2 + (2 if T <= 256 else 4) + 2 + 1 + (2 if side else 0)
+
+
+def dense_kernels(T: int, d: int, I: int, num_sms: int = 148) -> int:
+    """Launches of one moe_dense_swiglu: the offsets kernel, the two GEMMs,
+    and for each GEMM split over K (the library's rule: at most two waves of
+    pair tiles, 15 % or more fewer waves x K chunks) the kernel that sums
+    its partials."""
+    def splits(base, kit):
+        pairs = num_sms // 2
+        if base > 2 * pairs or kit < 4:
+            return 1
+        unsplit = -(-base // pairs) * kit
+        best, best_cost = 1, unsplit
+        for sp in range(2, min(8, kit // 2) + 1):
+            if -(-kit // sp) * (sp - 1) >= kit:
+                continue
+            cost = -(-(base * sp) // pairs) * -(-kit // sp)
+            if cost < best_cost:
+                best, best_cost = sp, cost
+        return best if best_cost * 100 <= unsplit * 85 else 1
+    n = 3
+    if T > 24 and d % 256 == 0 and I % 128 == 0:  # CTA-pair GEMMs
+        n += splits(-(-T // 256) * (I // 128), d // 128) > 1
+        n += splits(-(-T // 256) * (d // 256), I // 128) > 1
+    return n
 BWD_KERNELS = 11      # combine/router bwd (3), 4 grouped GEMMs (dW1 and dW3 in one), 2 gate GEMMs + split sum, un-permute
 BALANCE_KERNELS = 4   # balance partial sums, per-sequence f/P, loss, bias step
 # training-side balancing of the fwd+bwd step: sequences of the 8K pretraining
@@ -559,8 +585,8 @@ def measure(cfg, args, dev, world, rank, local):
            "e2e": {"value": e2e_value, "unit": "tokens/s",
                    "h2d_bytes_per_step": T * cfg.d * 2 * (2 if train else 1),
                    "d2h_bytes_per_step": T * cfg.d * 2},
-           "gpu_launches": (forward_kernels(T) + (BWD_KERNELS + BALANCE_KERNELS if train else 0))
-           * args.steps,
+           "gpu_launches": (forward_kernels(T, shared_on_side_stream(cfg, T, train))
+                            + (BWD_KERNELS + BALANCE_KERNELS if train else 0)) * args.steps,
            "config": config_dict(cfg, world, args.align, gemm_units(cfg, T, counts)["touched_experts"]),
            "n_phase": n_phase}
     if train:
@@ -771,7 +797,7 @@ def run_dense(args):
             "roofline": roof, "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
                     "d2h_bytes_per_step": T * d * 2},
-            "gpu_launches": 3 * args.steps}), flush=True)
+            "gpu_launches": dense_kernels(T, d, I) * args.steps}), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
     return 0
